@@ -1,0 +1,349 @@
+"""Pins for the float64 oracle: each check comes from something other than the
+oracle itself — the pages' worked example, a closed form, a library routine
+that computes the same definition, a brute-force twin, or an invariant.
+CPU only."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import ref, brute
+from workloads import normal, causal_mask_u8, alibi_slopes, cumulative
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+INT64_MAX = ref.INT64_MAX
+
+
+def f64(t):
+    return t.double().numpy()
+
+
+def rand(shape, seed):
+    return f64(normal(shape, "f32", seed))
+
+
+# ---------------------------------------------------------------------------
+# The pages' worked example (aclnnFlashAttentionVarLenScoreV5, call example).
+# ---------------------------------------------------------------------------
+
+def test_worked_example_sink_closed_form():
+    g = json.load(open(os.path.join(GOLDEN, "sink_example_tnd.json")))
+    t, n, d = g["T"], g["N"], g["D"]
+    one = torch.ones(t, n, d, dtype=torch.bfloat16)
+    res = ref.forward(f64(one), f64(one), f64(one), layout="TND", head_num=n,
+                      scale=g["scale"], atten_mask=np.zeros((t, t), np.uint8),
+                      pre_tokens=g["pre_tokens"], next_tokens=g["next_tokens"],
+                      sink=np.array([g["host_fill"]["sink"]]),
+                      actual_seq_q=g["actual_seq_q"], actual_seq_kv=g["actual_seq_kv"],
+                      softmax_out_layout=g["softmax_out_layout"])
+    exp = g["expected_without_rope"]
+    assert res["softmax_max"].shape == tuple(g["stats_shape"])
+    assert res["out"].shape == tuple(g["out_shape"])
+    np.testing.assert_allclose(res["softmax_max"], exp["softmax_max"], rtol=1e-12)
+    np.testing.assert_allclose(res["softmax_sum"], exp["softmax_sum"], rtol=1e-12)
+    np.testing.assert_allclose(res["out"], exp["out"], rtol=1e-12)
+    # the stored values are the closed form of the fixture's notes
+    s = g["scale"] * d
+    m = max(3.0, s)
+    l = t * math.exp(s - m) + math.exp(3.0 - m)
+    assert abs(exp["softmax_sum"] - l) < 1e-9 and abs(exp["out"] - t * math.exp(s - m) / l) < 1e-12
+    # rounded to bf16 the output is exactly 1.0
+    assert torch.tensor(res["out"]).to(torch.bfloat16).float().eq(1.0).all()
+
+
+# ---------------------------------------------------------------------------
+# Reduction to a library routine: torch scaled_dot_product_attention (float64).
+# ---------------------------------------------------------------------------
+
+def _sdpa(q, k, v, scale, bias):
+    """torch SDPA on one head with an additive float bias (-inf = excluded)."""
+    qt, kt, vt = (torch.from_numpy(x)[None, None] for x in (q, k, v))
+    b = torch.from_numpy(bias)[None, None]
+    out = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=b, scale=scale)
+    scores = scale * (torch.from_numpy(q) @ torch.from_numpy(k).T) + torch.from_numpy(bias)
+    return out[0, 0].numpy(), torch.logsumexp(scores, dim=-1).numpy()
+
+
+@pytest.mark.parametrize("sq,skv,d,dv,pre,nxt", [
+    (37, 53, 16, 16, INT64_MAX, INT64_MAX),
+    (64, 64, 32, 24, 10, 0),
+    (50, 70, 8, 8, 5, 30),
+])
+def test_head_matches_sdpa(sq, skv, d, dv, pre, nxt):
+    q, k, v = rand((sq, d), 1), rand((skv, d), 2), rand((skv, dv), 3)
+    pse = rand((sq, skv), 4)
+    rng = np.random.default_rng(5)
+    excluded = rng.random((sq, skv)) < 0.2
+    scale = 0.37
+    o, m, l = ref.head_forward(q, k, v, scale, pse=pse, excluded=excluded,
+                               pre_tokens=pre, next_tokens=nxt)
+    # the bias the test hands to SDPA: pse where kept, -inf where excluded by
+    # the mask or outside the band
+    i = np.arange(sq)[:, None]
+    j = np.arange(skv)[None, :]
+    outside = (j - i < -pre) | (j - i > nxt) | excluded
+    bias = np.where(outside, -np.inf, pse)
+    live = ~outside.all(axis=1)
+    o_ref, lse = _sdpa(q, k, v, scale, bias)
+    np.testing.assert_allclose(o[live], o_ref[live], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose((m + np.log(l))[live], lse[live], rtol=1e-12, atol=1e-12)
+
+
+def test_sink_matches_sdpa_with_extra_key():
+    """A sink is an extra key column with logit sink_n and a zero value row."""
+    sq, skv, d = 40, 33, 16
+    q, k, v = rand((sq, d), 11), rand((skv, d), 12), rand((skv, d), 13)
+    sink, scale = 1.7, 0.25
+    o, m, l = ref.head_forward(q, k, v, scale, sink=sink, next_tokens=0)
+    # extra key j = -1 placed first: q . 0 = 0, bias = sink, value 0
+    k2 = np.vstack([np.zeros((1, d)), k])
+    v2 = np.vstack([np.zeros((1, d)), v])
+    i = np.arange(sq)[:, None]
+    j = np.arange(skv)[None, :]
+    bias = np.hstack([np.full((sq, 1), sink), np.where(j - i > 0, -np.inf, 0.0)])
+    o_ref, lse = _sdpa(q, k2, v2, scale, bias)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(m + np.log(l), lse, rtol=1e-12)
+    assert (m >= sink).all()
+
+
+# ---------------------------------------------------------------------------
+# Brute force: the sink formula typed out with Python scalars.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("with_sink,with_pse,with_mask,pre,nxt", [
+    (False, False, False, INT64_MAX, INT64_MAX),
+    (True, False, False, INT64_MAX, 0),
+    (True, True, True, 2, 1),
+    (False, True, False, 1, -1),
+])
+def test_ref_matches_brute(with_sink, with_pse, with_mask, pre, nxt):
+    sq, skv, d, dv = 5, 4, 3, 2
+    q, k, v = rand((sq, d), 21), rand((skv, d), 22), rand((skv, dv), 23)
+    pse = rand((sq, skv), 24) if with_pse else None
+    excl = (np.random.default_rng(25).random((sq, skv)) < 0.3) if with_mask else None
+    sink = 0.4 if with_sink else None
+    o, m, l = ref.head_forward(q, k, v, 0.6, pse=pse, excluded=excl,
+                               pre_tokens=pre, next_tokens=nxt, sink=sink)
+    ob, mb, lb = brute.head_forward(q.tolist(), k.tolist(), v.tolist(), 0.6,
+                                    pse=None if pse is None else pse.tolist(),
+                                    excluded=None if excl is None else excl.tolist(),
+                                    pre_tokens=pre, next_tokens=nxt, sink=sink)
+    np.testing.assert_allclose(o, np.array(ob), rtol=1e-12, atol=1e-14)
+    np.testing.assert_array_equal(np.isinf(m), np.isinf(np.array(mb)))
+    fin = np.isfinite(m)
+    np.testing.assert_allclose(m[fin], np.array(mb)[fin], rtol=1e-13)
+    np.testing.assert_allclose(l, np.array(lb), rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Closed forms.
+# ---------------------------------------------------------------------------
+
+def test_constant_value_returns_constant():
+    q, k = rand((30, 8), 31), rand((45, 8), 32)
+    v = np.full((45, 5), 2.5)
+    o, _, _ = ref.head_forward(q, k, v, 0.3, next_tokens=3, pre_tokens=10)
+    np.testing.assert_allclose(o, 2.5, rtol=1e-13)
+
+
+def test_constant_value_with_sink():
+    q, k = rand((20, 8), 33), rand((20, 8), 34)
+    v = np.full((20, 3), -1.5)
+    o, m, l = ref.head_forward(q, k, v, 0.3, sink=0.8)
+    np.testing.assert_allclose(o, np.broadcast_to(-1.5 * (1.0 - np.exp(0.8 - m) / l)[:, None], o.shape), rtol=1e-12)
+
+
+def test_causal_first_row_is_v0():
+    q, k, v = rand((16, 8), 41), rand((16, 8), 42), rand((16, 8), 43)
+    o, m, l = ref.head_forward(q, k, v, 0.5, next_tokens=0)
+    np.testing.assert_allclose(o[0], v[0], rtol=1e-14)
+    assert l[0] == 1.0
+    np.testing.assert_allclose(m[0], 0.5 * q[0] @ k[0], rtol=1e-14)
+
+
+@pytest.mark.parametrize("sq,skv,pre,nxt", [
+    (40, 40, INT64_MAX, 0), (40, 40, 7, 0), (33, 50, 4, 9), (50, 20, 0, 0), (25, 25, 3, -2)])
+def test_zero_query_band_counts(sq, skv, pre, nxt):
+    """With Q = 0 and no pse every kept score is 0: m = 0, l = number of kept
+    keys = min(Skv-1, i+next) - max(0, i-pre) + 1 (inclusive band, top-left
+    aligned), and o = mean of the kept value rows."""
+    q = np.zeros((sq, 4))
+    k, v = rand((skv, 4), 51), rand((skv, 3), 52)
+    o, m, l = ref.head_forward(q, k, v, 1.0, pre_tokens=pre, next_tokens=nxt)
+    for i in range(sq):
+        lo = max(0, i - pre) if pre < INT64_MAX else 0
+        hi = min(skv - 1, i + nxt)
+        count = max(0, hi - lo + 1)
+        if count == 0:
+            assert m[i] == -np.inf and l[i] == 0 and (o[i] == 0).all()
+            continue
+        assert m[i] == 0.0 and l[i] == count
+        np.testing.assert_allclose(o[i], v[lo:hi + 1].mean(axis=0), rtol=1e-12, atol=1e-14)
+
+
+def test_alibi_geometric_series():
+    """Q = 0, ALiBi slope s, causal band of width pre: the kept weights are
+    r^0..r^K with r = e^-s and K = min(i, pre), so l = (1 - r^(K+1))/(1 - r)."""
+    sq, n_heads, pre = 64, 4, 9
+    slopes = f64(alibi_slopes(n_heads))
+    q = np.zeros((1, sq, n_heads, 8))
+    k, v = rand((1, sq, n_heads, 8), 61), rand((1, sq, n_heads, 8), 62)
+    res = ref.forward(q, k, v, layout="BSND", head_num=n_heads, scale=1.0,
+                      pse=slopes, pse_type=2, pre_tokens=pre, next_tokens=0)
+    for n in range(n_heads):
+        r = math.exp(-slopes[n])
+        for i in range(sq):
+            kk = min(i, pre)
+            l_exact = (1 - r ** (kk + 1)) / (1 - r)
+            assert res["softmax_max"][0, n, i, 0] == 0.0
+            np.testing.assert_allclose(res["softmax_sum"][0, n, i], l_exact, rtol=1e-13)
+
+
+def test_alibi_symmetric_band():
+    """Q = 0, ALiBi slope s, band [i - pre, i + next]: the kept weights are
+    r^|i-j|, so l = sum over the two one-sided geometric series
+    (1 - r^(a+1))/(1 - r) + r (1 - r^b)/(1 - r), a = min(i, pre),
+    b = min(S-1-i, next)."""
+    s, n_heads, pre, nxt = 40, 2, 6, 11
+    slopes = f64(alibi_slopes(n_heads))
+    q = np.zeros((1, n_heads, s, 8))
+    k, v = rand((1, n_heads, s, 8), 63), rand((1, n_heads, s, 8), 64)
+    res = ref.forward(q, k, v, layout="BNSD", head_num=n_heads, scale=1.0,
+                      pse=slopes, pse_type=2, pre_tokens=pre, next_tokens=nxt)
+    for n in range(n_heads):
+        r = math.exp(-slopes[n])
+        for i in range(s):
+            a, b = min(i, pre), min(s - 1 - i, nxt)
+            l_exact = (1 - r ** (a + 1)) / (1 - r) + r * (1 - r ** b) / (1 - r)
+            np.testing.assert_allclose(res["softmax_sum"][0, n, i], l_exact, rtol=1e-13)
+
+
+def test_empty_rows():
+    q, k, v = rand((6, 4), 71), rand((6, 4), 72), rand((6, 4), 73)
+    excl = np.zeros((6, 6), bool)
+    excl[2, :] = True
+    o, m, l = ref.head_forward(q, k, v, 1.0, excluded=excl)
+    assert (o[2] == 0).all() and m[2] == -np.inf and l[2] == 0
+    o, m, l = ref.head_forward(q, k, v, 1.0, excluded=excl, sink=-0.3)
+    assert (o[2] == 0).all() and m[2] == -0.3 and l[2] == 1.0
+    # a band that leaves row 0 empty (nextTokens < 0)
+    o, m, l = ref.head_forward(q, k, v, 1.0, pre_tokens=3, next_tokens=-1)
+    assert m[0] == -np.inf and l[0] == 0 and (o[0] == 0).all()
+
+
+def test_identity_value_exposes_probability_rows():
+    """With V = I the output row is the softmax row itself: it sums to 1, and
+    to 1 - e^(sink-m)/l with a sink."""
+    s = 24
+    q, k = rand((s, 8), 81), rand((s, 8), 82)
+    eye = np.eye(s)
+    o, m, l = ref.head_forward(q, k, eye, 0.4, next_tokens=0)
+    np.testing.assert_allclose(o.sum(axis=1), 1.0, rtol=1e-13)
+    assert (np.triu(o, 1) == 0).all()
+    assert (o >= 0).all() and ((l >= 1) & (l <= np.arange(1, s + 1))).all()
+    o, m, l = ref.head_forward(q, k, eye, 0.4, sink=0.9)
+    np.testing.assert_allclose(o.sum(axis=1), 1.0 - np.exp(0.9 - m) / l, rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Invariants across layouts, varlen, heads.
+# ---------------------------------------------------------------------------
+
+def _bnsd_to(x, layout):
+    if layout == "BNSD":
+        return x
+    if layout == "BSND":
+        return x.transpose(0, 2, 1, 3)
+    b, n, s, d = x.shape
+    if layout == "BSH":
+        return x.transpose(0, 2, 1, 3).reshape(b, s, n * d)
+    if layout == "SBH":
+        return x.transpose(2, 0, 1, 3).reshape(s, b, n * d)
+    raise ValueError(layout)
+
+
+def test_layouts_agree():
+    b, n, s, d = 2, 3, 21, 8
+    q, k, v = rand((b, n, s, d), 91), rand((b, n, s, d), 92), rand((b, n, s, d), 93)
+    sink = rand((n,), 94)
+    base = ref.forward(q, k, v, layout="BNSD", head_num=n, scale=0.3, next_tokens=0, sink=sink)
+    for layout in ("BSND", "BSH", "SBH"):
+        res = ref.forward(_bnsd_to(q, layout), _bnsd_to(k, layout), _bnsd_to(v, layout),
+                          layout=layout, head_num=n, scale=0.3, next_tokens=0, sink=sink)
+        np.testing.assert_array_equal(res["out"], _bnsd_to(base["out"], layout))
+        np.testing.assert_array_equal(res["softmax_max"], base["softmax_max"])
+        np.testing.assert_array_equal(res["softmax_sum"], base["softmax_sum"])
+
+
+def test_varlen_equals_each_sequence_alone():
+    lens, n, d = [5, 0, 17, 9], 2, 8
+    t = sum(lens)
+    q, k, v = rand((t, n, d), 101), rand((t, n, d), 102), rand((t, n, d), 103)
+    cum = cumulative(lens, leading_zero=False)
+    res = ref.forward(q, k, v, layout="TND", head_num=n, scale=0.5, next_tokens=0,
+                      actual_seq_q=cum, actual_seq_kv=cum, softmax_out_layout="same_as_input")
+    res_ntd = ref.forward(q, k, v, layout="TND", head_num=n, scale=0.5, next_tokens=0,
+                          actual_seq_q=cum, actual_seq_kv=cum)
+    np.testing.assert_array_equal(res_ntd["softmax_max"], res["softmax_max"].transpose(1, 0, 2))
+    start = 0
+    for length in lens:
+        if length:
+            sl = slice(start, start + length)
+            one = ref.forward(q[sl].transpose(1, 0, 2)[None], k[sl].transpose(1, 0, 2)[None],
+                              v[sl].transpose(1, 0, 2)[None], layout="BNSD", head_num=n,
+                              scale=0.5, next_tokens=0)
+            np.testing.assert_array_equal(res["out"][sl], one["out"][0].transpose(1, 0, 2))
+            np.testing.assert_array_equal(res["softmax_sum"][sl], one["softmax_sum"][0].transpose(1, 0, 2))
+        start += length
+
+
+def test_permuting_keys_leaves_output_unchanged():
+    q, k, v = rand((12, 8), 111), rand((19, 8), 112), rand((19, 6), 113)
+    perm = np.random.default_rng(114).permutation(19)
+    o1, m1, l1 = ref.head_forward(q, k, v, 0.7)
+    o2, m2, l2 = ref.head_forward(q, k[perm], v[perm], 0.7)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12)
+    np.testing.assert_allclose(m1, m2, rtol=1e-15)
+    np.testing.assert_allclose(l1, l2, rtol=1e-13)
+
+
+def test_gqa_equals_repeated_kv_heads():
+    b, nq, nkv, s, d = 1, 4, 2, 10, 8
+    q = rand((b, nq, s, d), 121)
+    k, v = rand((b, nkv, s, d), 122), rand((b, nkv, s, d), 123)
+    res = ref.forward(q, k, v, layout="BNSD", head_num=nq, scale=0.4)
+    rep = ref.forward(q, np.repeat(k, 2, axis=1), np.repeat(v, 2, axis=1), layout="BNSD",
+                      head_num=nq, scale=0.4)
+    np.testing.assert_array_equal(res["out"], rep["out"])
+
+
+def test_mask_tensor_broadcast_forms_agree():
+    b, n, s, d = 2, 2, 9, 4
+    q, k, v = rand((b, n, s, d), 131), rand((b, n, s, d), 132), rand((b, n, s, d), 133)
+    m2 = causal_mask_u8(s, s).numpy()
+    outs = []
+    for mask in (m2, m2[None, None], np.broadcast_to(m2, (b, 1, s, s)), np.broadcast_to(m2, (b, n, s, s))):
+        outs.append(ref.forward(q, k, v, layout="BNSD", head_num=n, scale=0.5, atten_mask=mask)["out"])
+    band = ref.forward(q, k, v, layout="BNSD", head_num=n, scale=0.5, next_tokens=0)["out"]
+    for o in outs:
+        np.testing.assert_array_equal(o, band)
+
+
+def test_forward_rows_matches_forward():
+    b, n, s, d = 2, 3, 30, 8
+    q, k, v = rand((b, s, n, d), 141), rand((b, s, n, d), 142), rand((b, s, n, d), 143)
+    sink = rand((n,), 144)
+    full = ref.forward(q, k, v, layout="BSND", head_num=n, scale=0.3, pre_tokens=6,
+                       next_tokens=0, sink=sink)
+    rows = [(0, 0, 0), (1, 2, 29), (0, 1, 17)]
+    o, m, l = ref.forward_rows(q, k, v, rows, layout="BSND", head_num=n, scale=0.3,
+                               pre_tokens=6, next_tokens=0, sink=sink)
+    for r, (bb, nn, i) in enumerate(rows):
+        # a one-row product may round differently from the blocked one
+        np.testing.assert_allclose(o[r], full["out"][bb, i, nn], rtol=1e-13, atol=1e-15)
+        np.testing.assert_allclose(m[r], full["softmax_max"][bb, nn, i, 0], rtol=1e-14)
+        np.testing.assert_allclose(l[r], full["softmax_sum"][bb, nn, i, 0], rtol=1e-13)
