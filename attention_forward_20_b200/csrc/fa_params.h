@@ -1,0 +1,75 @@
+// Launch parameters shared by the host planner (api.cpp) and the kernels.
+// Internal to the library; the public ABI is include/fa_fwd.h.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+// Row addressing.  For every operand, element (b, n, i, d) of a sequence lives
+// at  base + b*stride_b + n*stride_n + (seq_off_b + i)*stride_s + d
+// where seq_off_b is the sequence's first token for the packed TND layout
+// (from the cumulative lengths) and 0 otherwise (stride_b is 0 for TND).
+struct FaParams {
+    const void* q;
+    const void* k;
+    const void* v;
+    void* o;
+    float* smax;
+    float* ssum;
+    const void* pse;      // dense bias (query dtype) or fp32 ALiBi slopes
+    const uint8_t* mask;  // nonzero = excluded; read only when mask_on
+    const float* sink;    // fp32 [Nq] or nullptr
+
+    int64_t q_b, q_n, q_s;
+    int64_t k_b, k_n, k_s;
+    int64_t v_b, v_n, v_s;
+    int64_t o_b, o_n, o_s;
+    int64_t st_b, st_n, st_s;       // statistics; the 8 lanes are contiguous
+    int64_t pse_b, pse_n, pse_i;    // dense bias strides (column stride 1); ALiBi: pse_b, pse_n
+    int64_t mask_b, mask_n, mask_i; // mask strides (column stride 1), broadcast dims have 0
+
+    const int64_t* cu_q;   // device, [B+1] with a leading 0 (TND only)
+    const int64_t* cu_kv;
+
+    int32_t B, Nq, Nkv, group;  // group = Nq / Nkv
+    int32_t D, Dv;
+    int32_t Sq, Skv;            // sequence lengths (TND: the longest)
+    int32_t pre, next;          // band, clamped to +-(Sq + Skv + 1)
+    float scale;                // scaleValue in fp32
+    float scale_log2;           // scaleValue * log2(e) in fp32 (tcgen05 path)
+    int32_t pse_type;           // 0 none, 1 dense, 2 ALiBi slopes
+    int32_t mask_on;
+    int32_t has_sink;
+    int32_t varlen;
+    int32_t dtype;              // FA_F32 / FA_F16 / FA_BF16
+
+    // tcgen05 path: persistent schedule
+    int32_t n_items;            // work items of (b, n, 256-row query block)
+    int32_t n_qb;               // query blocks per (b, n) for the dense layouts
+    int32_t items_per_n_block;  // dense: B * Nq
+    const int4* table;          // TND: {b, qb, q_len, kv_len} per (sequence, block), heads implied
+    int32_t table_len;
+    int32_t neg_scale;          // scaleValue < 0: the kernel negates K inside the MMA
+    int32_t Tq, Tkv;            // rows of the query / key tensors (TND: packed tokens; else Sq / Skv)
+    int32_t mask_cols;          // allocated width of a mask row (columns readable from mask)
+    int32_t o_vec;              // output rows allow 16-byte stores
+    int32_t mask_vec;           // mask rows allow 16-byte loads
+    int32_t pse_vec;            // dense bias rows allow 16-byte loads
+};
+
+enum KernelKind { KERNEL_SIMT = 0, KERNEL_SM100 = 1 };
+
+// Tensor-map descriptors (CUtensorMap is 128 bytes, 64-byte aligned).
+struct alignas(64) TmaDesc {
+    uint64_t opaque[16];
+};
+
+cudaError_t launch_simt(const FaParams& p, cudaStream_t stream);
+cudaError_t launch_sm100(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk,
+                         const TmaDesc& tv, int num_sms, cudaStream_t stream);
+// Encodes the Q/K/V tensor maps for the tcgen05 kernel.
+cudaError_t make_sm100_tmaps(const FaParams& p, TmaDesc* tq, TmaDesc* tk, TmaDesc* tv);
+uint64_t read_and_clear_device_error(cudaError_t* err);
+
+}  // namespace fa

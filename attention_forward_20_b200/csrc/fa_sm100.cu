@@ -1,0 +1,741 @@
+// tcgen05 attention forward for sm_100a (fp16 / bf16 inputs, head dim 64 or 128).
+//
+// What it computes is the forward and sink formulas of the
+// aclnnFlashAttentionVarLenScoreV5 page ("计算公式"), tiled with the
+// FlashAttention online softmax (aclnnFlashAttentionScore, "功能描述").
+//
+// One persistent CTA per SM walks a static list of work items; an item is one
+// (batch, query head, 256-row query block), split into two 128-row query tiles
+// that ping-pong on the tensor core:
+//
+//   warps 0-3  softmax tile 0   (thread r owns TMEM lane r = query row r)
+//   warps 4-7  softmax tile 1
+//   warp  8    TMA producer     (Q tiles, then K and V 128-row blocks into a ring)
+//   warp  9    MMA issuer       (S = Q·Kᵀ and O += P·V with tcgen05.mma)
+//
+// TMEM (512 columns): S_t at columns [128t, 128t+128) as fp32; P_t (fp16/bf16,
+// two per column) overwrites the first 64 of them and is the A operand of
+// P·V; O_t at [256 + t*D, 256 + (t+1)*D) as fp32.
+//
+// Softmax runs in the log2 domain: x = s * scale * log2(e) (+ bias * log2(e)),
+// p = 2^(x - m_used).  The running row max m_run is exact; m_used, the max the
+// exponentials are taken against, only moves (rescaling l and O) when m_run
+// exceeds it by more than 8, so that p <= 2^8 and most blocks skip the O
+// rescale.  The epilogue folds in the sink (max and denominator) and converts
+// the statistics back to natural-log units.
+//
+// Every wait is bounded (mbar_wait): on a timeout the CTA records the failure
+// in a device error word, drains its in-flight copies and MMAs, frees TMEM and
+// exits.
+#include "fa_params.h"
+#include "sm100_ptx.cuh"
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <math_constants.h>
+
+#include <mutex>
+#include <type_traits>
+
+namespace fa {
+
+__device__ unsigned long long g_fa_error;
+
+namespace {
+using namespace ptx;
+
+constexpr int kTileM = 128;     // query rows per tile (one TMEM lane each)
+constexpr int kTileN = 128;     // keys per block
+constexpr int kQBlock = 256;    // query rows per work item (two tiles)
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kHeadGroup = 16;  // heads whose items run together, so their K/V stay in L2
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.69314718055994531f;
+constexpr float kRescaleThreshold = 8.0f;
+
+// wait sites recorded in the error word
+enum : int {
+    kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull,
+    kSiteSFull, kSiteOFull, kSiteDrain
+};
+
+template <int D>
+struct Cfg {
+    static constexpr int kChunks = D / 64;             // 128-byte swizzle chunks per row
+    static constexpr int kChunkBytes = kTileM * 128;   // one chunk of a 128-row tile
+    static constexpr int kTileBytes = kTileM * D * 2;  // one Q, K or V tile
+    static constexpr int kStages = (D == 128) ? 4 : 8; // K/V ring slots
+    static constexpr int kSmemBytes = (2 + kStages) * kTileBytes + 1024;
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kOCol = 256;
+};
+
+struct Barriers {
+    uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2];
+    uint64_t kv_full[8], kv_empty[8];
+    uint64_t drain;
+};
+
+struct Item {
+    int b, n, nk, qb, q_len, kv_len;
+    int64_t q_off, kv_off;
+};
+
+// Work item -> (batch, head, query block).  Dense layouts: groups of
+// kHeadGroup heads; inside a group the query blocks go from the last (the
+// most keys under a causal band) to the first, heads fastest.  TND: the host
+// table lists (sequence, block) longest first; heads fastest.
+__device__ __forceinline__ Item decode_item(const FaParams& p, int item) {
+    Item it;
+    if (p.varlen) {
+        const int e = item / p.Nq;
+        it.n = item - e * p.Nq;
+        const int4 t = p.table[e];
+        it.b = t.x;
+        it.qb = t.y;
+        it.q_len = t.z;
+        it.kv_len = t.w;
+        it.q_off = p.cu_q[it.b];
+        it.kv_off = p.cu_kv[it.b];
+    } else {
+        const int bn_total = p.B * p.Nq;
+        const int per_group = kHeadGroup * p.n_qb;
+        const int g = item / per_group;
+        const int within = item - g * per_group;
+        const int g_heads = min(kHeadGroup, bn_total - g * kHeadGroup);
+        const int level = within / g_heads;
+        const int bn = g * kHeadGroup + (within - level * g_heads);
+        it.qb = p.n_qb - 1 - level;
+        it.b = bn / p.Nq;
+        it.n = bn - it.b * p.Nq;
+        it.q_len = p.Sq;
+        it.kv_len = p.Skv;
+        it.q_off = 0;
+        it.kv_off = 0;
+    }
+    it.nk = it.n / p.group;
+    return it;
+}
+
+// Key blocks [lo, hi] that query tile t of the item touches under the band
+// -pre <= j - i <= next; lo > hi when none.  `valid` says the tile has rows.
+struct TileRange {
+    int valid, lo, hi;
+    __device__ __forceinline__ bool active() const { return valid && hi >= lo; }
+    __device__ __forceinline__ bool has(int jb) const { return valid && jb >= lo && jb <= hi; }
+};
+
+__device__ __forceinline__ TileRange tile_range(const FaParams& p, const Item& it, int t) {
+    TileRange r{0, 0, -1};
+    const int r0 = it.qb * kQBlock + t * kTileM;
+    if (r0 >= it.q_len) return r;
+    r.valid = 1;
+    const int r1 = min(it.q_len, r0 + kTileM) - 1;
+    const int j_lo = max(0, r0 - p.pre);
+    const int j_hi = min(it.kv_len - 1, r1 + p.next);
+    if (j_hi >= j_lo) {
+        r.lo = j_lo / kTileN;
+        r.hi = j_hi / kTileN;
+    }
+    return r;
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int site) {
+    const bool ok = mbar_wait(bar, parity, abort, site);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// ---------------------------------------------------------------------------
+// TMA producer (one thread)
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
+                             const CUtensorMap* tv, uint8_t* sQ, uint8_t* sKV, Barriers& bars,
+                             volatile int* abort) {
+    using C = Cfg<D>;
+    uint32_t kv_fill = 0, q_fill[2] = {0, 0};
+    bool ok = true;
+
+    auto load_tile = [&](const CUtensorMap* tm, uint8_t* dst, uint64_t* bar, int row, int head, int b,
+                         int64_t seq_off) {
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c) {
+            if (p.varlen)
+                tma_load_3d(dst + c * C::kChunkBytes, tm, bar, c * 64, (int)(seq_off + row), head);
+            else
+                tma_load_4d(dst + c * C::kChunkBytes, tm, bar, c * 64, row, head, b);
+        }
+    };
+
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const Item it = decode_item(p, item);
+        const TileRange tr[2] = {tile_range(p, it, 0), tile_range(p, it, 1)};
+        if (!tr[0].active() && !tr[1].active()) continue;
+        const int lo = tr[0].active() ? (tr[1].active() ? min(tr[0].lo, tr[1].lo) : tr[0].lo) : tr[1].lo;
+        const int hi = tr[0].active() ? (tr[1].active() ? max(tr[0].hi, tr[1].hi) : tr[0].hi) : tr[1].hi;
+
+        auto load_q = [&](int t) -> bool {
+            if (!mbar_wait(&bars.q_empty[t], (q_fill[t] & 1) ^ 1, abort, kSiteQEmpty)) return false;
+            mbar_arrive_expect_tx(&bars.q_full[t], C::kTileBytes);
+            load_tile(tq, sQ + t * C::kTileBytes, &bars.q_full[t], it.qb * kQBlock + t * kTileM, it.n, it.b,
+                      it.q_off);
+            ++q_fill[t];
+            return true;
+        };
+        auto load_kv = [&](const CUtensorMap* tm, int jb) -> bool {
+            const int slot = kv_fill % C::kStages;
+            if (!mbar_wait(&bars.kv_empty[slot], ((kv_fill / C::kStages) & 1) ^ 1, abort, kSiteKvEmpty))
+                return false;
+            mbar_arrive_expect_tx(&bars.kv_full[slot], C::kTileBytes);
+            load_tile(tm, sKV + slot * C::kTileBytes, &bars.kv_full[slot], jb * kTileN, it.nk, it.b, it.kv_off);
+            ++kv_fill;
+            return true;
+        };
+
+        if (tr[0].active() && !load_q(0)) { ok = false; break; }
+        for (int jb = lo; ok && jb <= hi; ++jb) {
+            if (!load_kv(tk, jb)) { ok = false; break; }
+            if (jb == lo && tr[1].active() && !load_q(1)) { ok = false; break; }
+            if (!load_kv(tv, jb)) { ok = false; break; }
+        }
+    }
+
+    // Drain: the latest fill of every slot (and Q buffer) must have landed
+    // before the CTA may exit; earlier fills of a slot completed before the
+    // slot could be refilled.
+    for (int s = 0; s < C::kStages; ++s) {
+        if ((uint32_t)s < kv_fill) {
+            const uint32_t last = kv_fill - 1 - ((kv_fill - 1 - s) % C::kStages);
+            mbar_wait(&bars.kv_full[s], (last / C::kStages) & 1, abort, kSiteDrain);
+        }
+    }
+    for (int t = 0; t < 2; ++t)
+        if (q_fill[t]) mbar_wait(&bars.q_full[t], (q_fill[t] - 1) & 1, abort, kSiteDrain);
+}
+
+// ---------------------------------------------------------------------------
+// MMA issuer (one thread)
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& bars, uint32_t tmem,
+                        volatile int* abort) {
+    using C = Cfg<D>;
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    const uint32_t idesc_qk = idesc_f16(kBf16, kTileM, kTileN, false, false, p.neg_scale != 0);
+    constexpr uint32_t idesc_pv = idesc_f16(kBf16, kTileM, D, false, true, false);
+    uint32_t kv_use = 0, q_use[2] = {0, 0}, p_cnt[2] = {0, 0};
+    bool ok = true;
+
+    auto wait_kv = [&](int* slot) -> bool {
+        *slot = kv_use % C::kStages;
+        const bool r = mbar_wait(&bars.kv_full[*slot], (kv_use / C::kStages) & 1, abort, kSiteKvFull);
+        ++kv_use;
+        return r;
+    };
+    // S_t = Q_t · K^T: D/16 MMAs of K = 16; both operands K-major, 128-byte
+    // swizzled, 8-row groups 1024 bytes apart, 64-column chunks one tile-chunk apart.
+    auto issue_qk = [&](int t, int slot) {
+        const uint32_t qa = smem_u32(sQ + t * C::kTileBytes);
+        const uint32_t ka = smem_u32(sKV + slot * C::kTileBytes);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k >> 2) * C::kChunkBytes + (k & 3) * 32;
+            mma_ss(tmem + t * kTileN, sdesc_sw128(qa + off, 1024, 16), sdesc_sw128(ka + off, 1024, 16), idesc_qk,
+                   k > 0 ? 1u : 0u);
+        }
+    };
+    // O_t (+)= P_t · V: 8 MMAs of K = 16 keys; P from TMEM (8 columns per step),
+    // V MN-major: 8-key groups 1024 bytes apart, 64-column chunks kChunkBytes apart.
+    auto issue_pv = [&](int t, int slot, bool accumulate) {
+        const uint32_t va = smem_u32(sKV + slot * C::kTileBytes);
+#pragma unroll
+        for (int k = 0; k < kTileN / 16; ++k) {
+            mma_ts(tmem + C::kOCol + t * D, tmem + t * kTileN + k * 8, sdesc_sw128(va + k * 2048, 1024, C::kChunkBytes),
+                   idesc_pv, (k > 0 || accumulate) ? 1u : 0u);
+        }
+    };
+
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const Item it = decode_item(p, item);
+        const TileRange tr[2] = {tile_range(p, it, 0), tile_range(p, it, 1)};
+        if (!tr[0].active() && !tr[1].active()) continue;
+        const int lo = tr[0].active() ? (tr[1].active() ? min(tr[0].lo, tr[1].lo) : tr[0].lo) : tr[1].lo;
+        const int hi = tr[0].active() ? (tr[1].active() ? max(tr[0].hi, tr[1].hi) : tr[0].hi) : tr[1].hi;
+
+        for (int t = 0; t < 2; ++t)
+            if (tr[t].active() && !mbar_wait(&bars.q_full[t], q_use[t] & 1, abort, kSiteQFull)) ok = false;
+        int sk;
+        if (!ok || !wait_kv(&sk)) { ok = false; break; }
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t) {
+            if (tr[t].has(lo)) {
+                issue_qk(t, sk);
+                tc_commit(&bars.s_full[t]);
+                if (lo == tr[t].hi) tc_commit(&bars.q_empty[t]);
+            }
+        }
+        tc_commit(&bars.kv_empty[sk]);
+
+        for (int jb = lo; jb <= hi; ++jb) {
+            int sv, sk2 = 0;
+            const bool has_next = jb < hi;
+            if (!wait_kv(&sv) || (has_next && !wait_kv(&sk2))) { ok = false; break; }
+            tc_fence_after();
+            for (int t = 0; t < 2; ++t) {
+                if (tr[t].has(jb)) {
+                    if (!mbar_wait(&bars.p_full[t], p_cnt[t] & 1, abort, kSitePFull)) { ok = false; break; }
+                    ++p_cnt[t];
+                    tc_fence_after();
+                    issue_pv(t, sv, jb != tr[t].lo);
+                    if (jb == tr[t].hi) tc_commit(&bars.o_full[t]);
+                }
+                if (has_next && tr[t].has(jb + 1)) {
+                    issue_qk(t, sk2);
+                    tc_commit(&bars.s_full[t]);
+                    if (jb + 1 == tr[t].hi) tc_commit(&bars.q_empty[t]);
+                }
+            }
+            if (!ok) break;
+            tc_commit(&bars.kv_empty[sv]);
+            if (has_next) tc_commit(&bars.kv_empty[sk2]);
+        }
+        for (int t = 0; t < 2; ++t)
+            if (tr[t].active()) ++q_use[t];
+    }
+    // Drain: every MMA this thread issued completes before TMEM is freed.
+    tc_commit(&bars.drain);
+    mbar_wait(&bars.drain, 0, abort, kSiteDrain);
+}
+
+// ---------------------------------------------------------------------------
+// Softmax warpgroup t (128 threads; thread r owns query row r of the tile)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float a, float b);
+template <>
+__device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+template <>
+__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Additive bias of 8 consecutive keys starting at j from a dense pse row (query dtype), times log2(e).
+template <typename T>
+__device__ __forceinline__ void load_bias8(const T* row, int j, int kv_len, bool vec, float* out) {
+    if (vec && j + 8 <= kv_len) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + j));
+        const T* h = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) out[e] = to_f(h[e]) * kLog2e;
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) out[e] = (j + e < kv_len) ? to_f(row[j + e]) * kLog2e : 0.f;
+    }
+}
+
+// Excluded flags (nonzero) of 16 consecutive keys starting at j from a mask row.
+__device__ __forceinline__ uint32_t load_mask16(const uint8_t* row, int j, int cols, bool vec) {
+    uint32_t bits = 0;
+    if (vec && j + 16 <= cols) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + j));
+        const uint8_t* b = reinterpret_cast<const uint8_t*>(&u);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) bits |= (b[e] != 0 ? 1u : 0u) << e;
+    } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if (j + e < cols && row[j + e] != 0) bits |= 1u << e;
+    }
+    return bits;
+}
+
+template <typename T, int D, bool kBias>
+__device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, volatile int* abort, int t) {
+    using C = Cfg<D>;
+    const int quad = (threadIdx.x >> 5) & 3;
+    const int row = quad * 32 + (threadIdx.x & 31);
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * kTileN;
+    const uint32_t tO = tmem + lane_off + C::kOCol + t * D;
+    const float sl2 = p.scale_log2;
+    uint32_t s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const Item it = decode_item(p, item);
+        const TileRange tr = tile_range(p, it, t);
+        if (!tr.valid) continue;
+        const int r0 = it.qb * kQBlock + t * kTileM;
+        const int i = r0 + row;
+        const bool row_ok = i < it.q_len;
+
+        float slope_l2 = 0.f;
+        const T* pse_row = nullptr;
+        if (kBias) {
+            if (p.pse_type == 2)
+                slope_l2 = static_cast<const float*>(p.pse)[it.b * p.pse_b + it.n * p.pse_n] * kLog2e;
+            else if (row_ok)
+                pse_row = static_cast<const T*>(p.pse) + it.b * p.pse_b + it.n * p.pse_n + (int64_t)i * p.pse_i;
+        }
+        const uint8_t* mask_row =
+            (p.mask_on && row_ok) ? p.mask + it.b * p.mask_b + it.n * p.mask_n + (int64_t)i * p.mask_i : nullptr;
+
+        float m_run = -CUDART_INF_F, m_used = -CUDART_INF_F, l = 0.f;
+        for (int jb = tr.lo; jb <= tr.hi; ++jb) {
+            if (!warp_wait(&bars.s_full[t], s_cnt & 1, abort, kSiteSFull)) { ok = false; break; }
+            ++s_cnt;
+            tc_fence_after();
+            float s[128];
+            {
+                uint32_t sr[128];
+                tmem_ld_x128(tS, sr);
+#pragma unroll
+                for (int c = 0; c < kTileN; ++c) s[c] = __uint_as_float(sr[c]);
+            }
+            const int j0 = jb * kTileN;
+            const bool full = !p.mask_on && (j0 + kTileN <= it.kv_len) && (j0 - (r0 + kTileM - 1) >= -p.pre) &&
+                              (j0 + kTileN - 1 - r0 <= p.next);
+
+            // scores in the log2 domain (bias path) and the block's row max
+            float m_blk;
+            if constexpr (kBias) {
+                const float fi = (float)(i - j0);
+#pragma unroll
+                for (int c8 = 0; c8 < kTileN; c8 += 8) {
+                    float bias[8];
+                    if (p.pse_type == 2) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) bias[e] = -slope_l2 * fabsf(fi - (float)(c8 + e));
+                    } else if (pse_row) {
+                        load_bias8(pse_row, j0 + c8, it.kv_len, p.pse_vec != 0, bias);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) bias[e] = 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) s[c8 + e] = fmaf(s[c8 + e], sl2, bias[e]);
+                }
+            }
+            if (!full) {
+#pragma unroll
+                for (int c16 = 0; c16 < kTileN; c16 += 16) {
+                    const uint32_t excl = mask_row ? load_mask16(mask_row, j0 + c16, p.mask_cols, p.mask_vec != 0) : 0u;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int j = j0 + c16 + e;
+                        const int d = j - i;
+                        const bool keep = j < it.kv_len && d >= -p.pre && d <= p.next && !((excl >> e) & 1u);
+                        if (!keep) s[c16 + e] = -CUDART_INF_F;
+                    }
+                }
+            }
+            {
+                float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+#pragma unroll
+                for (int c = 4; c < kTileN; c += 4) {
+                    m0 = fmaxf(m0, s[c]);
+                    m1 = fmaxf(m1, s[c + 1]);
+                    m2 = fmaxf(m2, s[c + 2]);
+                    m3 = fmaxf(m3, s[c + 3]);
+                }
+                m_blk = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+                if constexpr (!kBias) m_blk *= sl2;
+            }
+
+            const float m_new = fmaxf(m_run, m_blk);
+            const bool need = (m_new - m_used) > kRescaleThreshold;  // false while both are -inf
+            const float alpha = need ? ex2(m_used - m_new) : 1.f;    // 0 when m_used is -inf
+            if (jb > tr.lo && __any_sync(0xffffffffu, need)) {
+                // O_t is stable: the commit behind this block's S_t covered the last P·V.
+#pragma unroll
+                for (int cc = 0; cc < D; cc += 32) {
+                    uint32_t o[32];
+                    tmem_ld_x32(tO + cc, o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st_x32(tO + cc, o);
+                }
+            }
+            if (need) {
+                l *= alpha;
+                m_used = m_new;
+            }
+            m_run = m_new;
+            const float shift = (m_used == -CUDART_INF_F) ? 0.f : m_used;
+
+            float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+            uint32_t pk[64];
+#pragma unroll
+            for (int c = 0; c < kTileN; c += 4) {
+                float e0, e1, e2, e3;
+                if constexpr (kBias) {
+                    e0 = ex2(s[c] - shift);
+                    e1 = ex2(s[c + 1] - shift);
+                    e2 = ex2(s[c + 2] - shift);
+                    e3 = ex2(s[c + 3] - shift);
+                } else {
+                    e0 = ex2(fmaf(s[c], sl2, -shift));
+                    e1 = ex2(fmaf(s[c + 1], sl2, -shift));
+                    e2 = ex2(fmaf(s[c + 2], sl2, -shift));
+                    e3 = ex2(fmaf(s[c + 3], sl2, -shift));
+                }
+                l0 += e0;
+                l1 += e1;
+                l2 += e2;
+                l3 += e3;
+                pk[c / 2] = pack2<T>(e0, e1);
+                pk[c / 2 + 1] = pack2<T>(e2, e3);
+            }
+            l += (l0 + l1) + (l2 + l3);
+            tmem_st_x64(tS, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars.p_full[t]);
+        }
+        if (!ok) break;
+
+        // ---- epilogue: sink, normalisation, statistics ----------------------
+        const bool has_blocks = tr.hi >= tr.lo;
+        if (has_blocks) {
+            if (!warp_wait(&bars.o_full[t], o_cnt & 1, abort, kSiteOFull)) { ok = false; break; }
+            ++o_cnt;
+            tc_fence_after();
+        }
+        float m_f = m_run, l_f, o_scale;
+        if (p.has_sink) {
+            const float sk = p.sink[it.n] * kLog2e;
+            m_f = fmaxf(m_run, sk);
+            const float a = (m_used == -CUDART_INF_F) ? 0.f : ex2(m_used - m_f);
+            l_f = l * a + ex2(sk - m_f);
+            o_scale = a / l_f;
+        } else {
+            l_f = l * ((m_used == -CUDART_INF_F) ? 0.f : ex2(m_used - m_run));
+            o_scale = (l > 0.f) ? 1.f / l : 0.f;
+        }
+
+        T* orow = static_cast<T*>(p.o) + it.b * p.o_b + it.n * p.o_n + (it.q_off + i) * p.o_s;
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32) {
+            uint32_t o[32];
+            if (has_blocks) {
+                tmem_ld_x32(tO + cc, o);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] = 0u;
+            }
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                w[e] = pack2<T>(__uint_as_float(o[2 * e]) * o_scale, __uint_as_float(o[2 * e + 1]) * o_scale);
+            if (row_ok) {
+                if (p.o_vec) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + cc);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                } else {
+                    uint32_t* dst = reinterpret_cast<uint32_t*>(orow + cc);
+                    if ((reinterpret_cast<uintptr_t>(dst) & 3u) == 0) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) dst[e] = w[e];
+                    } else {
+                        const T* h = reinterpret_cast<const T*>(w);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) orow[cc + e] = h[e];
+                    }
+                }
+            }
+        }
+        if (row_ok) {
+            const int64_t so = it.b * p.st_b + it.n * p.st_n + (it.q_off + i) * p.st_s;
+            const float m_nat = m_f * kLn2;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                p.smax[so + e] = m_nat;
+                p.ssum[so + e] = l_f;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel
+// ---------------------------------------------------------------------------
+template <typename T, int D, bool kBias>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_v, const FaParams p) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = smem;
+    uint8_t* sKV = smem + 2 * C::kTileBytes;
+    __shared__ Barriers bars;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bars.q_full[t], 1);
+            mbar_init(&bars.q_empty[t], 1);
+            mbar_init(&bars.s_full[t], 1);
+            mbar_init(&bars.p_full[t], kTileM);
+            mbar_init(&bars.o_full[t], 1);
+        }
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&bars.kv_full[s], 1);
+            mbar_init(&bars.kv_empty[s], 1);
+        }
+        mbar_init(&bars.drain, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kLoadWarp && lane == 0) {
+        prefetch_tmap(&tmap_q);
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_v);
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(&tmem_base, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+
+    if (warp < 8) {
+        run_softmax<T, D, kBias>(p, bars, tmem, &abort_flag, warp >> 2);
+    } else if (warp == kLoadWarp) {
+        if (lane == 0) run_producer<D>(p, &tmap_q, &tmap_k, &tmap_v, sQ, sKV, bars, &abort_flag);
+        __syncwarp();
+    } else {
+        if (lane == 0) run_mma<T, D>(p, sQ, sKV, bars, tmem, &abort_flag);
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, C::kTmemCols);
+    if (threadIdx.x == 0 && abort_flag != 0)
+        atomicCAS(&g_fa_error, 0ull, (static_cast<unsigned long long>(abort_flag) << 32) | (blockIdx.x + 1u));
+}
+
+template <typename T, int D, bool kBias>
+cudaError_t launch_t(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, const TmaDesc& tv, int num_sms,
+                     cudaStream_t stream) {
+    using C = Cfg<D>;
+    auto kern = fa_fwd_sm100_kernel<T, D, kBias>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int grid = p.n_items < num_sms ? p.n_items : num_sms;
+    if (grid <= 0) return cudaSuccess;
+    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(*reinterpret_cast<const CUtensorMap*>(&tq),
+                                                    *reinterpret_cast<const CUtensorMap*>(&tk),
+                                                    *reinterpret_cast<const CUtensorMap*>(&tv), p);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_d(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, const TmaDesc& tv, int num_sms,
+                     cudaStream_t stream) {
+    const bool bias = p.pse_type != 0;
+    if (p.D == 128)
+        return bias ? launch_t<T, 128, true>(p, tq, tk, tv, num_sms, stream)
+                    : launch_t<T, 128, false>(p, tq, tk, tv, num_sms, stream);
+    return bias ? launch_t<T, 64, true>(p, tq, tk, tv, num_sms, stream)
+                : launch_t<T, 64, false>(p, tq, tk, tv, num_sms, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Tensor maps (host)
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// Byte stride of a dimension; a size-1 dimension's stride never matters, so
+// any legal value (16) stands in for it.
+cuuint64_t stride_bytes(int64_t elems, int64_t size) {
+    return size == 1 ? 16 : static_cast<cuuint64_t>(elems) * 2;
+}
+
+// Box of 64 columns (128 bytes, the swizzle span) x 128 rows; 128-byte swizzle;
+// out-of-range rows read as zero.
+cudaError_t encode(TmaDesc* out, const FaParams& p, const void* base, int rows, int heads, int64_t s_stride,
+                   int64_t n_stride, int64_t b_stride) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const CUtensorMapDataType dt = p.dtype == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r;
+    if (p.varlen) {
+        const cuuint64_t dims[3] = {(cuuint64_t)p.D, (cuuint64_t)rows, (cuuint64_t)heads};
+        const cuuint64_t strides[2] = {stride_bytes(s_stride, rows), stride_bytes(n_stride, heads)};
+        const cuuint32_t box[3] = {64, 128, 1};
+        const cuuint32_t es[3] = {1, 1, 1};
+        r = fn(reinterpret_cast<CUtensorMap*>(out), dt, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+        const cuuint64_t dims[4] = {(cuuint64_t)p.D, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)p.B};
+        const cuuint64_t strides[3] = {stride_bytes(s_stride, rows), stride_bytes(n_stride, heads),
+                                       stride_bytes(b_stride, p.B)};
+        const cuuint32_t box[4] = {64, 128, 1, 1};
+        const cuuint32_t es[4] = {1, 1, 1, 1};
+        r = fn(reinterpret_cast<CUtensorMap*>(out), dt, 4, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t make_sm100_tmaps(const FaParams& p, TmaDesc* tq, TmaDesc* tk, TmaDesc* tv) {
+    cudaError_t e = encode(tq, p, p.q, p.Tq, p.Nq, p.q_s, p.q_n, p.q_b);
+    if (e == cudaSuccess) e = encode(tk, p, p.k, p.Tkv, p.Nkv, p.k_s, p.k_n, p.k_b);
+    if (e == cudaSuccess) e = encode(tv, p, p.v, p.Tkv, p.Nkv, p.v_s, p.v_n, p.v_b);
+    return e;
+}
+
+cudaError_t launch_sm100(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, const TmaDesc& tv, int num_sms,
+                         cudaStream_t stream) {
+    if (p.dtype == 2) return launch_d<__nv_bfloat16>(p, tq, tk, tv, num_sms, stream);
+    return launch_d<__half>(p, tq, tk, tv, num_sms, stream);
+}
+
+uint64_t read_and_clear_device_error(cudaError_t* err) {
+    unsigned long long word = 0, zero = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&word, g_fa_error, sizeof(word));
+    if (e == cudaSuccess && word) e = cudaMemcpyToSymbol(g_fa_error, &zero, sizeof(zero));
+    if (err) *err = e;
+    return word;
+}
+
+}  // namespace fa

@@ -1,0 +1,391 @@
+"""Throughput of the attention forward on B200: one JSON line on rank 0.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload C] [--impl reference]
+
+A step is one forward over the workload's whole batch (every step of the hot
+path runs in one kernel launch).  The default workload is the dense BNSD fp16
+forward B=2, N=24, S=4096, D=128.  Under torchrun each rank runs its own shard
+of a batch N times as large (independent sequences, no data-path collective:
+weak scaling); the time is the max over ranks of the summed per-step CUDA-event
+times, and L2 is flushed (256 MiB write) before every step.
+
+--impl reference times the float64 CPU oracle (rank 0 only) on a bounded
+sample of the same workload with the same metric.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import build  # noqa: E402
+
+METRIC = "FA forward TFLOP/s and % of B200 dense BF16/FP16 peak (1 GPU)"
+UNIT = "TFLOP/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ["attention_forward_20_b200/csrc/fa_sm100.cu", "attention_forward_20_b200/csrc/sm100_ptx.cuh"]
+L2_FLUSH_BYTES = 256 << 20
+
+
+def workload_desc(w):
+    lens = {"BNSD": (w.q.shape[0], w.q.shape[2]), "BSND": (w.q.shape[0], w.q.shape[1]),
+            "BSH": (w.q.shape[0], w.q.shape[1]), "SBH": (w.q.shape[1], w.q.shape[0])}
+    d = w.q.shape[-1] if w.layout not in ("BSH", "SBH") else w.q.shape[-1] // w.head_num
+    cfg = {"workload": f"{w.name} {w.layout} {w.dtype}", "layout": w.layout, "dtype": w.dtype,
+           "heads": w.head_num, "head_dim": d}
+    if w.layout == "TND":
+        cfg.update(tokens=w.q.shape[0], lengths=w.extra.get("lengths"))
+    else:
+        b, s = lens[w.layout]
+        cfg.update(batch=b, seq_len=s)
+    if w.next_tokens == 0:
+        cfg["mask"] = "causal" + (f" band preTokens={w.pre_tokens}" if w.pre_tokens < 2**62 else "")
+    if w.pse_type == 2:
+        cfg["pse"] = "ALiBi slopes in-kernel"
+    if w.sink is not None:
+        cfg["sink"] = "per-head fp32"
+    return cfg
+
+
+def tile_flops(w):
+    """4 * D * (query-row x key pairs), counted over every 128x128 tile that
+    holds at least one kept pair (the headline rule), and the exact kept-pair
+    FLOPs beside it."""
+    d = w.q.shape[-1] if w.layout not in ("BSH", "SBH") else w.q.shape[-1] // w.head_num
+    if w.layout == "TND":
+        lens_q = np.diff([0] + list(w.actual_seq_q))
+        lens_k = np.diff([0] + list(w.actual_seq_kv))
+        seqs = list(zip(lens_q, lens_k))
+    else:
+        b = w.q.shape[1] if w.layout == "SBH" else w.q.shape[0]
+        sq = {"BNSD": w.q.shape[2], "BSND": w.q.shape[1], "BSH": w.q.shape[1], "SBH": w.q.shape[0]}[w.layout]
+        skv = {"BNSD": w.k.shape[2], "BSND": w.k.shape[1], "BSH": w.k.shape[1], "SBH": w.k.shape[0]}[w.layout]
+        seqs = [(sq, skv)] * b
+    pre, nxt = w.pre_tokens, w.next_tokens
+    tiles = exact = 0
+    for sq, skv in seqs:
+        for i0 in range(0, sq, 128):
+            i1 = min(sq, i0 + 128) - 1
+            for j0 in range(0, skv, 128):
+                j1 = min(skv, j0 + 128) - 1
+                # kept pairs of this tile: j in [max(j0, i-pre), min(j1, i+next)] per row i
+                rows = np.arange(i0, i1 + 1)
+                lo = np.maximum(j0, rows - min(pre, 2**40))
+                hi = np.minimum(j1, rows + min(nxt, 2**40))
+                kept = np.clip(hi - lo + 1, 0, None).sum()
+                if kept:
+                    tiles += 128 * 128
+                    exact += int(kept)
+    heads = w.head_num
+    return 4.0 * d * tiles * heads, 4.0 * d * exact * heads
+
+
+def sources_sha():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            peaks = json.load(f)
+        return float(peaks["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst; fp16 nominal ratio 1)"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback 1.59 PFLOP/s"
+
+
+def load_traffic(workload_name):
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = t.get(workload_name)
+    if not entry or entry.get("kernel_sources_sha") != sources_sha():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML in a thread."""
+
+    REASONS = {
+        0x0000000000000008: "hw_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000004: "sw_power_cap",
+    }
+
+    def __init__(self, device_index, interval=0.002):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.interval = interval
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def fa_kwargs(w, dev):
+    c = lambda t: None if t is None else t.to(dev)  # noqa: E731
+    pse = c(w.pse)
+    return dict(input_layout=w.layout, head_num=w.head_num, scale=w.scale, real_shift=pse,
+                pse_type=w.pse_type if pse is not None else None, atten_mask=c(w.atten_mask),
+                mask_mode=w.mask_mode, sink=c(w.sink), actual_seq_qlen=w.actual_seq_q,
+                actual_seq_kvlen=w.actual_seq_kv, pre_tokens=w.pre_tokens, next_tokens=w.next_tokens,
+                softmax_out_layout=w.softmax_out_layout)
+
+
+def time_oracle(w, budget_s, max_heads=None):
+    """Float64 oracle on whole (batch, head) pairs of the workload until
+    `budget_s` seconds have passed; returns (flops done, seconds, heads done)."""
+    from oracle import ref
+    d = w.q.shape[-1] if w.layout not in ("BSH", "SBH") else w.q.shape[-1] // w.head_num
+    qh = ref.heads_view(w.q.double().numpy(), w.layout, d)
+    kh = ref.heads_view(w.k.double().numpy(), w.layout, d)
+    vh = ref.heads_view(w.v.double().numpy(), w.layout, d)
+    n_kv = kh.shape[1]
+    group = w.head_num // n_kv
+    sink = None if w.sink is None else w.sink.double().numpy()
+    pse = None if w.pse is None else w.pse.double().numpy()
+    if w.layout == "TND":
+        cq = [0] + list(w.actual_seq_q)
+        ck = [0] + list(w.actual_seq_kv)
+        pairs = [(b, n) for b in range(len(cq) - 1) for n in range(w.head_num)]
+    else:
+        pairs = [(b, n) for b in range(qh.shape[0]) for n in range(w.head_num)]
+    flops = secs = 0.0
+    heads = 0
+    for (b, n) in pairs[:max_heads]:
+        if w.layout == "TND":
+            q, k, v = (qh[cq[b]:cq[b + 1], n], kh[ck[b]:ck[b + 1], n // group], vh[ck[b]:ck[b + 1], n // group])
+        else:
+            q, k, v = qh[b, n], kh[b, n // group], vh[b, n // group]
+        rows = np.arange(q.shape[0])
+        t0 = time.perf_counter()
+        ref.head_forward(q, k, v, w.scale, rows=rows,
+                         pse=ref._pse_rows(pse, w.pse_type, b, n, rows, k.shape[0]),
+                         pre_tokens=w.pre_tokens, next_tokens=w.next_tokens,
+                         sink=None if sink is None else sink[n])
+        secs += time.perf_counter() - t0
+        flops += 4.0 * d * q.shape[0] * k.shape[0]
+        heads += 1
+        if secs >= budget_s:
+            break
+    return flops, secs, heads
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    w = build(args.workload)
+    for _ in range(args.warmup):
+        time_oracle(w, 0.0, max_heads=1)
+    flops = secs = 0.0
+    heads = 0
+    for _ in range(args.steps):
+        f, s, h = time_oracle(w, 0.0, max_heads=1)
+        flops, secs, heads = flops + f, secs + s, heads + h
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_desc(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"one whole (batch, head) of the workload per step, {heads} heads"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import attention_forward_20_b200 as fa
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    # each rank: its own shard (seed offset by rank) of the workload's batch
+    w = build(args.workload)
+    if rank:
+        g = torch.Generator().manual_seed(1000003 * rank)
+        for name in ("q", "k", "v"):
+            t = getattr(w, name)
+            setattr(w, name, torch.randn(t.shape, generator=g, dtype=torch.float32).to(t.dtype))
+    flops_tiles, flops_exact = tile_flops(w)
+    q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
+    kw = fa_kwargs(w, dev)
+    out, smax, ssum = fa.fa_fwd(q, k, v, **kw)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.fa_fwd(q, k, v, out=out, softmax_max=smax, softmax_sum=ssum, **kw)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    kernel_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    status, word = fa.device_error()
+    if status != 0:
+        raise SystemExit(f"kernel error word {word:#x}")
+
+    # end to end: pinned host inputs -> device, forward, result -> pinned host
+    host = [t.pin_memory() for t in (w.q, w.k, w.v)]
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    host_sm = torch.empty(smax.shape, dtype=smax.dtype).pin_memory()
+    host_ss = torch.empty(ssum.shape, dtype=ssum.dtype).pin_memory()
+    dq, dk, dv = (torch.empty_like(t, device=dev) for t in host)
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        for d_, h_ in zip((dq, dk, dv), host):
+            d_.copy_(h_, non_blocking=True)
+        fa.fa_fwd(dq, dk, dv, out=out, softmax_max=smax, softmax_sum=ssum, **kw)
+        host_out.copy_(out, non_blocking=True)
+        host_sm.copy_(smax, non_blocking=True)
+        host_ss.copy_(ssum, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = sum(t.numel() * t.element_size() for t in (host_out, host_sm, host_ss))
+
+    t = torch.tensor([kernel_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    kernel_ms, e2e_ms = float(t[0]), float(t[1])
+    if dist:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    ms_per_step = kernel_ms / args.steps
+    value = flops_tiles * world / (ms_per_step * 1e-3) / 1e12
+    per_gpu = flops_tiles / (ms_per_step * 1e-3) / 1e12
+    peak, peak_src = load_peak()
+    traffic = load_traffic(w.name)
+    fl, secs, heads = time_oracle(w, args.cpu_budget)
+    cpu_value = fl / secs / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": dict(workload_desc(w), parallelism=f"dp{world} (independent shards)",
+                       l2="flushed before every step (256 MiB write); inputs 201 MB > 126 MB L2",
+                       flops_tile_counted=flops_tiles, flops_exact=flops_exact,
+                       pct_of_nominal_2250=100.0 * per_gpu / 2250.0),
+        "roofline": {"bound": "tensor", "achieved": per_gpu, "peak": peak, "unit": UNIT,
+                     "frac": per_gpu / peak, "traffic": traffic, "peak_source": peak_src},
+        "cpu_baseline": {"value": cpu_value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"{heads} whole (batch, head) pairs of the workload, float64 NumPy, "
+                                   f"{secs:.1f} s"},
+        "e2e": {"value": flops_tiles * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

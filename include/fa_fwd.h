@@ -1,0 +1,170 @@
+/*
+ * fa_fwd.h — C ABI of the B200 (sm_100a) FlashAttention self-attention forward.
+ *
+ * The operation (aclnnFlashAttentionVarLenScoreV5 page, "计算公式": the forward
+ * formula and the sink formula; aclnnFlashAttentionScore page, parameter list):
+ *
+ *   for every batch b and query head n, with i a query row and j a key row of
+ *   that sequence:
+ *     s_ij    = scaleValue * <q_i, k_j> + pse_ij
+ *     keep_ij = (-preTokens <= j - i <= nextTokens) && !attenMask_ij
+ *     m_i     = max({s_ij : keep_ij} U {sink_n})
+ *     l_i     = sum_keep exp(s_ij - m_i) + exp(sink_n - m_i)
+ *     out_i   = sum_keep exp(s_ij - m_i) v_j / l_i
+ *   softmaxMax_i = m_i (natural-log units), softmaxSum_i = l_i, each written to
+ *   all 8 lanes of the trailing axis.  The sink terms are absent without a
+ *   sink.  A row with nothing kept gets out = 0, m = -inf, l = 0 (with a sink:
+ *   out = 0, m = sink_n, l = 1).
+ *
+ * Two-stage call, as on both operator pages ("接口原型" / "函数原型"):
+ *   1. fa_fwd_get_workspace_size() validates every argument on the host, plans
+ *      the launch and returns the device workspace size and an executor.  It
+ *      makes no CUDA call and touches no device memory.
+ *   2. fa_fwd() enqueues the work on `stream` and consumes the executor.
+ *
+ * All floating-point accumulation is fp32.  Q·Kᵀ and P·V run on the tcgen05
+ * tensor cores for fp16/bf16 inputs with head dim 64 or 128; fp32 inputs (and
+ * any other head dim up to 256) run on an exact-FFMA CUDA-core kernel.
+ */
+#ifndef FA_FWD_H
+#define FA_FWD_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------------------
+ * Status codes.  The first three carry the numbers of the pages' aclnn return
+ * codes (aclnnFlashAttentionScore "返回值"; aclnnFlashAttentionVarLenScoreV5
+ * return-code table).  The rest are this library's own.
+ * ------------------------------------------------------------------------- */
+typedef int32_t fa_status;
+#define FA_SUCCESS 0
+#define FA_ERR_PARAM_NULLPTR 161001   /* a required input, output or out-pointer is NULL      */
+#define FA_ERR_PARAM_INVALID 161002   /* a dtype or a layout/format string is not supported   */
+#define FA_ERR_INNER_NULLPTR 561103   /* a shape or attribute is out of the supported range   */
+#define FA_ERR_CUDA 561200            /* a CUDA runtime call or the kernel launch failed      */
+#define FA_ERR_WORKSPACE 561201       /* workspace smaller than fa_fwd_get_workspace_size said */
+#define FA_ERR_DEVICE_TIMEOUT 561202  /* a kernel wait ran past its limit (see fa_device_error) */
+
+/* Element types of fa_tensor.dtype. */
+#define FA_F32 0
+#define FA_F16 1
+#define FA_BF16 2
+#define FA_U8 3
+#define FA_BOOL 4
+
+/* Position-bias kinds for pseType (the pages leave pseType's values undefined;
+ * these are this library's). */
+#define FA_PSE_NONE 0   /* realShift must be NULL (1 is also accepted with NULL) */
+#define FA_PSE_DENSE 1  /* realShift [B or 1, N or 1, Sq, Skv], query dtype, added after scaling */
+#define FA_PSE_ALIBI 2  /* realShift fp32 slopes [N] or [B, N]: pse_ij = -slope * |i - j|     */
+
+/* Mask modes for maskMode (the pages' sparseMode numbering is defined in a
+ * section they do not include; these are this library's). */
+#define FA_MASK_TENSOR 0  /* attenMask, when given, is read element by element, and the band applies */
+#define FA_MASK_BAND 1    /* the caller asserts attenMask equals the preTokens/nextTokens band; the
+                             kernel does not read attenMask and skips tiles outside the band */
+
+/* A strided tensor view.  `data` is a device pointer, borrowed (the caller owns
+ * the memory and keeps it valid until the work on the stream has finished).
+ * Strides count elements, not bytes.  The innermost stride must be 1.  Up to 8
+ * dimensions. */
+typedef struct fa_tensor {
+    void* data;
+    int32_t dtype;
+    int32_t ndim;
+    int64_t shape[8];
+    int64_t strides[8];
+} fa_tensor;
+
+/* Opaque plan made by stage 1 (aclOpExecutor on the pages). */
+typedef struct fa_executor fa_executor;
+
+/* Stage 1.  Validates, plans, and reports the workspace size.
+ *
+ * query / key / value: device tensors, dtype FA_F32, FA_F16 or FA_BF16 (all
+ *   three equal), layout `inputLayout`:
+ *     "BNSD" [B, N, S, D]   "BSND" [B, S, N, D]   "BSH" [B, S, N*D]
+ *     "SBH"  [S, B, N*D]    "TND"  [T, N, D] (T = sequences packed back to back)
+ *   key/value may have fewer heads than query (Nq % Nkv == 0; query head n
+ *   reads key/value head n / (Nq/Nkv)).  value's head dim may be smaller than
+ *   the query/key head dim.
+ * realShift: optional bias, see FA_PSE_*; NULL for none.
+ * attenMask: optional FA_U8/FA_BOOL, nonzero = excluded.  Shapes [B,N,Sq,Skv],
+ *   [B,1,Sq,Skv], [1,1,Sq,Skv] or [Sq,Skv]; with "TND" only [Sq,Skv] indexed by
+ *   in-sequence positions (Sq, Skv at least the longest sequence).
+ * sink: optional fp32 [headNum], one logit per query head, not scaled.
+ * actualSeqQLen / actualSeqKvLen: host int64 arrays of nSeqQ == nSeqKv == B
+ *   entries, cumulative lengths without a leading 0 ([2,2,0,2,2] is passed as
+ *   [2,4,4,6,8]); required with "TND", must be NULL otherwise; the last entry
+ *   equals T of query (resp. key/value).  Zero-length sequences are allowed.
+ * scaleValue: finite and nonzero.  keepProb: must be 1.0 (no dropout).
+ * preTokens / nextTokens: the band -preTokens <= j - i <= nextTokens, inclusive,
+ *   counted from the start of each sequence; INT64_MAX for no bound.
+ *   preTokens + nextTokens must be >= 0.
+ * headNum: N of query, 1..256.  innerPrecise: 0, 1 or 2 (accepted; the
+ *   arithmetic is always fp32 and empty rows always get the defined values).
+ * maskMode: FA_MASK_TENSOR or FA_MASK_BAND.  pseType: FA_PSE_*.
+ * softmaxOutLayout: NULL/"" or "same_as_input".  With "TND" the statistics are
+ *   [N, T, 8] for "" and [T, N, 8] for "same_as_input"; other layouts always
+ *   use [B, N, Sq, 8].
+ * softmaxMax / softmaxSum: fp32 outputs of that shape.  attentionOut: query's
+ *   dtype and layout with value's head dim.
+ * workspaceSize / executor: out-pointers.  On success *executor owns host
+ *   memory until fa_fwd() or fa_executor_destroy() releases it.
+ *
+ * Returns FA_SUCCESS, FA_ERR_PARAM_NULLPTR, FA_ERR_PARAM_INVALID or
+ * FA_ERR_INNER_NULLPTR; on error *executor is set to NULL.  Thread-safe; no
+ * CUDA call is made. */
+FA_API fa_status fa_fwd_get_workspace_size(
+    const fa_tensor* query, const fa_tensor* key, const fa_tensor* value,
+    const fa_tensor* realShift, const fa_tensor* attenMask, const fa_tensor* sink,
+    const int64_t* actualSeqQLen, int64_t nSeqQ,
+    const int64_t* actualSeqKvLen, int64_t nSeqKv,
+    double scaleValue, double keepProb, int64_t preTokens, int64_t nextTokens,
+    int64_t headNum, const char* inputLayout, int64_t innerPrecise,
+    int64_t maskMode, int64_t pseType, const char* softmaxOutLayout,
+    const fa_tensor* softmaxMax, const fa_tensor* softmaxSum, const fa_tensor* attentionOut,
+    uint64_t* workspaceSize, fa_executor** executor);
+
+/* Stage 2.  Enqueues the forward on `stream` (a cudaStream_t; NULL = the
+ * legacy default stream) on the current device and returns without waiting.
+ * `workspace` is caller-owned device memory of at least the size stage 1
+ * returned (NULL allowed when that size is 0); it must stay untouched until
+ * the stream work has finished.  The executor is consumed and freed on every
+ * return path, success or error.
+ * Returns FA_SUCCESS, FA_ERR_PARAM_NULLPTR (executor NULL, or workspace NULL
+ * with a nonzero size), FA_ERR_WORKSPACE or FA_ERR_CUDA. */
+FA_API fa_status fa_fwd(void* workspace, uint64_t workspaceSize, fa_executor* executor, void* stream);
+
+/* Releases an executor that will not be passed to fa_fwd().  NULL is a no-op. */
+FA_API void fa_executor_destroy(fa_executor* executor);
+
+/* Static description of the plan ("kernel=... grid=... items=..."), valid
+ * while the executor lives.  For logging and tests. */
+FA_API const char* fa_executor_describe(const fa_executor* executor);
+
+/* Reads and clears the current device's kernel error word.  Every wait in the
+ * tcgen05 kernel has a time limit; a wait that runs out records an error
+ * here and the kernel returns early instead of hanging.  Synchronises the
+ * device.  Returns FA_SUCCESS, FA_ERR_DEVICE_TIMEOUT or FA_ERR_CUDA; when
+ * `detail` is not NULL it receives the raw word (0 when clean). */
+FA_API fa_status fa_device_error(uint64_t* detail);
+
+/* Human-readable name of a status code (static string). */
+FA_API const char* fa_status_string(fa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_FWD_H */

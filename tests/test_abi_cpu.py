@@ -1,0 +1,311 @@
+"""The C ABI on the CPU: the library loads, exports every function that
+include/fa_fwd.h declares, and stage 1 validates arguments with the status
+codes of the aclnn operator pages (161001 / 161002 / 561103).  Stage 1 makes no
+CUDA call, so host tensors stand in for device ones here."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import attention_forward_20_b200 as fa
+from attention_forward_20_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa_fwd.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from attention_forward_20_b200 import build
+    build.build()
+    return _abi.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_documented_entry_points():
+    assert declared_functions() == sorted(_abi.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(built):
+    for name in declared_functions():
+        assert hasattr(built, name), name
+    out = os.popen(f"nm -D --defined-only {_abi.LIB_PATH}").read()
+    exported = set(re.findall(r" T (fa_\w+)", out))
+    assert set(declared_functions()) <= exported
+    # nothing else leaks out of the library's own namespace
+    assert {s for s in exported if s.startswith("fa_")} == set(declared_functions())
+
+
+def test_status_strings():
+    for code in (fa.FA_SUCCESS, fa.FA_ERR_PARAM_NULLPTR, fa.FA_ERR_PARAM_INVALID, fa.FA_ERR_INNER_NULLPTR,
+                 fa.FA_ERR_CUDA, fa.FA_ERR_WORKSPACE, fa.FA_ERR_DEVICE_TIMEOUT):
+        assert str(code) in _abi.status_string(code) or code == 0
+    assert _abi.status_string(12345) == "unknown fa_status"
+
+
+def qkv(shape, dtype=torch.float16):
+    return [torch.zeros(shape, dtype=dtype) for _ in range(3)]
+
+
+def plan(q, k, v, **kw):
+    kw.setdefault("input_layout", "BNSD")
+    kw.setdefault("head_num", q.shape[1] if kw["input_layout"] == "BNSD" else None)
+    return fa.plan(q, k, v, **kw)
+
+
+# ---------------------------------------------------------------------------
+# Stage 1 accepts the five workloads and picks the kernel
+# ---------------------------------------------------------------------------
+
+def test_plan_tiny_fp32_uses_cuda_core_kernel():
+    q, k, v = qkv((1, 2, 128, 64), torch.float32)
+    st, ws, text = plan(q, k, v, scale=0.125)
+    assert st == 0 and ws == 0 and "kernel=simt_fp32acc" in text
+
+
+@pytest.mark.parametrize("layout,shape,n,dtype,d", [
+    ("BNSD", (2, 24, 256, 128), 24, torch.float16, 128),
+    ("BSND", (2, 256, 8, 128), 8, torch.bfloat16, 128),
+    ("BSH", (2, 512, 1024), 16, torch.float16, 64),
+    ("SBH", (300, 2, 256), 4, torch.bfloat16, 64),
+])
+def test_plan_half_types_use_tcgen05(layout, shape, n, dtype, d):
+    q, k, v = qkv(shape, dtype)
+    st, ws, text = fa.plan(q, k, v, input_layout=layout, head_num=n)
+    assert st == 0, _abi.status_string(st)
+    assert "kernel=sm100_tcgen05" in text and f"D={d}" in text and ws == 0
+
+
+def test_plan_varlen_workspace_holds_lengths_and_table():
+    lens = [400, 1069, 1344, 763, 931, 1380, 1693, 612]
+    cum = [sum(lens[:i + 1]) for i in range(len(lens))]
+    q, k, v = qkv((8192, 24, 128), torch.bfloat16)
+    st, ws, text = fa.plan(q, k, v, input_layout="TND", head_num=24, actual_seq_qlen=cum,
+                           actual_seq_kvlen=cum, next_tokens=0)
+    assert st == 0
+    blocks = sum((x + 255) // 256 for x in lens)
+    assert "kernel=sm100_tcgen05" in text and f"items={blocks * 24}" in text
+    cu_bytes = (2 * (len(lens) + 1) * 8 + 255) // 256 * 256
+    assert ws == cu_bytes + blocks * 16
+
+
+def test_plan_unaligned_stride_falls_to_cuda_core_kernel():
+    base = torch.zeros(2, 4, 100, 130, dtype=torch.float16)
+    q = base[..., :128]  # row stride 130 elements = 260 bytes: not a TMA stride
+    st, _, text = fa.plan(q, q, q, input_layout="BNSD", head_num=4)
+    assert st == 0 and "kernel=simt_fp32acc" in text
+
+
+# ---------------------------------------------------------------------------
+# 161001: NULL required arguments
+# ---------------------------------------------------------------------------
+
+def raw_stage1(q, k, v, out, smax, ssum, layout=b"BNSD", head_num=2, drop=()):
+    lib = _abi.load()
+    ts = {name: fa._ft(t) for name, t in dict(q=q, k=k, v=v, out=out, smax=smax, ssum=ssum).items()}
+    for name in drop:
+        ts[name] = None
+    p = lambda t: ctypes.byref(t) if t is not None else None  # noqa: E731
+    ws = ctypes.c_uint64(0)
+    ex = ctypes.c_void_p(None)
+    st = lib.fa_fwd_get_workspace_size(p(ts["q"]), p(ts["k"]), p(ts["v"]), None, None, None, None, 0, None, 0,
+                                       0.125, 1.0, _abi.INT64_MAX, _abi.INT64_MAX, head_num, layout, 0, 0, 0, b"",
+                                       p(ts["smax"]), p(ts["ssum"]), p(ts["out"]), ctypes.byref(ws),
+                                       ctypes.byref(ex))
+    if st == 0:
+        lib.fa_executor_destroy(ex)
+    else:
+        assert ex.value is None
+    return st
+
+
+def small():
+    q, k, v = qkv((1, 2, 16, 64))
+    out = torch.zeros_like(q)
+    smax = torch.zeros(1, 2, 16, 8)
+    ssum = torch.zeros(1, 2, 16, 8)
+    return q, k, v, out, smax, ssum
+
+
+def test_valid_raw_call_succeeds():
+    assert raw_stage1(*small()) == 0
+
+
+@pytest.mark.parametrize("name", ["q", "k", "v", "out", "smax", "ssum"])
+def test_null_required_tensor(name):
+    assert raw_stage1(*small(), drop=(name,)) == fa.FA_ERR_PARAM_NULLPTR
+
+
+def test_null_out_pointers():
+    lib = _abi.load()
+    q, k, v, out, smax, ssum = [fa._ft(t) for t in small()]
+    r = ctypes.byref
+    st = lib.fa_fwd_get_workspace_size(r(q), r(k), r(v), None, None, None, None, 0, None, 0, 0.125, 1.0,
+                                       _abi.INT64_MAX, _abi.INT64_MAX, 2, b"BNSD", 0, 0, 0, b"", r(smax), r(ssum),
+                                       r(out), None, None)
+    assert st == fa.FA_ERR_PARAM_NULLPTR
+
+
+def test_fa_fwd_null_executor_and_small_workspace():
+    lib = _abi.load()
+    assert lib.fa_fwd(None, 0, None, None) == fa.FA_ERR_PARAM_NULLPTR
+    lens = [5, 7]
+    q, k, v = qkv((12, 2, 64))
+    out = torch.zeros_like(q)
+    smax = torch.zeros(2, 12, 8)
+    ssum = torch.zeros(2, 12, 8)
+    status, ws, ex = fa._stage1(q, k, v, out, smax, ssum, input_layout="TND", head_num=2, scale=0.1,
+                                real_shift=None, pse_type=0, atten_mask=None, mask_mode=0, sink=None,
+                                actual_seq_qlen=[5, 12], actual_seq_kvlen=[5, 12], pre_tokens=_abi.INT64_MAX,
+                                next_tokens=_abi.INT64_MAX, keep_prob=1.0, inner_precise=0, softmax_out_layout="")
+    assert status == 0 and ws > 0
+    # too small a workspace is refused before any CUDA call, and the executor is consumed
+    assert lib.fa_fwd(ctypes.c_void_p(16), ctypes.c_uint64(ws - 1), ex, None) == fa.FA_ERR_WORKSPACE
+    del lens
+
+
+# ---------------------------------------------------------------------------
+# 161002: dtypes and format strings
+# ---------------------------------------------------------------------------
+
+def test_bad_layout_string():
+    assert raw_stage1(*small(), layout=b"NSD") == fa.FA_ERR_PARAM_INVALID
+
+
+def test_mixed_qkv_dtypes():
+    q, k, v, out, smax, ssum = small()
+    assert raw_stage1(q, k.to(torch.bfloat16), v, out, smax, ssum) == fa.FA_ERR_PARAM_INVALID
+
+
+def test_out_dtype_and_stats_dtype():
+    q, k, v, out, smax, ssum = small()
+    assert raw_stage1(q, k, v, out.float(), smax, ssum) == fa.FA_ERR_PARAM_INVALID
+    assert raw_stage1(q, k, v, out, smax.half(), ssum) == fa.FA_ERR_PARAM_INVALID
+
+
+def test_integer_inputs_rejected():
+    q, k, v, out, smax, ssum = small()
+    i8 = [t.to(torch.uint8) for t in (q, k, v, out)]
+    assert raw_stage1(*i8, smax, ssum) == fa.FA_ERR_PARAM_INVALID
+
+
+def test_bad_mask_and_sink_dtypes():
+    q, k, v = qkv((1, 2, 16, 64))
+    st, _, _ = plan(q, k, v, atten_mask=torch.zeros(16, 16, dtype=torch.float16))
+    assert st == fa.FA_ERR_PARAM_INVALID
+    st, _, _ = plan(q, k, v, sink=torch.zeros(2, dtype=torch.float16))
+    assert st == fa.FA_ERR_PARAM_INVALID
+
+
+def test_bad_softmax_out_layout():
+    q, k, v = qkv((1, 2, 16, 64))
+    assert plan(q, k, v, softmax_out_layout="NTD")[0] == fa.FA_ERR_PARAM_INVALID
+    out = torch.zeros_like(q)
+    s = torch.zeros(1, 2, 16, 8)
+    status, _, _ = fa._stage1(q, k, v, out, s, s.clone(), input_layout="BNSD", head_num=2, scale=0.1,
+                              real_shift=None, pse_type=0, atten_mask=None, mask_mode=0, sink=None,
+                              actual_seq_qlen=None, actual_seq_kvlen=None, pre_tokens=_abi.INT64_MAX,
+                              next_tokens=_abi.INT64_MAX, keep_prob=1.0, inner_precise=0, softmax_out_layout="NTD")
+    assert status == fa.FA_ERR_PARAM_INVALID
+
+
+# ---------------------------------------------------------------------------
+# 561103: shapes and attributes
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kw", [
+    dict(keep_prob=0.9),
+    dict(scale=0.0),
+    dict(scale=float("inf")),
+    dict(inner_precise=3),
+    dict(mask_mode=2),
+    dict(pre_tokens=3, next_tokens=-4),
+    dict(pse_type=2),  # ALiBi without slopes
+])
+def test_bad_attributes(kw):
+    q, k, v = qkv((1, 2, 16, 64))
+    st, _, _ = plan(q, k, v, **kw)
+    assert st == fa.FA_ERR_INNER_NULLPTR
+
+
+def test_head_num_range_and_mismatch():
+    q, k, v = qkv((1, 2, 16, 64))
+    assert plan(q, k, v, head_num=3)[0] == fa.FA_ERR_INNER_NULLPTR
+    q, k, v = qkv((1, 257, 4, 64))
+    assert plan(q, k, v, head_num=257)[0] == fa.FA_ERR_INNER_NULLPTR
+
+
+def test_gqa_ratio():
+    q = torch.zeros(1, 6, 16, 64, dtype=torch.float16)
+    kv = torch.zeros(1, 4, 16, 64, dtype=torch.float16)
+    assert plan(q, kv, kv)[0] == fa.FA_ERR_INNER_NULLPTR
+    kv = torch.zeros(1, 3, 16, 64, dtype=torch.float16)
+    st, _, text = plan(q, kv, kv)
+    assert st == 0 and "Nkv=3" in text
+
+
+def test_head_dim_limits():
+    q, k, v = qkv((1, 2, 16, 320))
+    assert plan(q, k, v)[0] == fa.FA_ERR_INNER_NULLPTR
+    q, k, _ = qkv((1, 2, 16, 64))
+    v = torch.zeros(1, 2, 16, 96, dtype=torch.float16)  # value head dim above key's
+    assert plan(q, k, v)[0] == fa.FA_ERR_INNER_NULLPTR
+    v = torch.zeros(1, 2, 16, 32, dtype=torch.float16)  # below is allowed (CUDA-core kernel)
+    st, _, text = plan(q, k, v)
+    assert st == 0 and "simt" in text
+
+
+def test_batch_and_seq_mismatch():
+    q = torch.zeros(2, 2, 16, 64, dtype=torch.float16)
+    k = torch.zeros(1, 2, 16, 64, dtype=torch.float16)
+    assert plan(q, k, k)[0] == fa.FA_ERR_INNER_NULLPTR
+    k = torch.zeros(2, 2, 16, 64, dtype=torch.float16)
+    v = torch.zeros(2, 2, 17, 64, dtype=torch.float16)
+    assert plan(q, k, v)[0] == fa.FA_ERR_INNER_NULLPTR
+
+
+def test_varlen_arguments():
+    q, k, v = qkv((12, 2, 64))
+    base = dict(input_layout="TND", head_num=2)
+    assert plan(q, k, v, **base)[0] == fa.FA_ERR_PARAM_NULLPTR               # TND needs lengths
+    assert plan(q, k, v, **base, actual_seq_qlen=[5, 12], actual_seq_kvlen=[12])[0] == fa.FA_ERR_INNER_NULLPTR
+    assert plan(q, k, v, **base, actual_seq_qlen=[7, 5, 12], actual_seq_kvlen=[7, 5, 12])[0] == \
+        fa.FA_ERR_INNER_NULLPTR                                                # not cumulative
+    assert plan(q, k, v, **base, actual_seq_qlen=[5, 11], actual_seq_kvlen=[5, 11])[0] == \
+        fa.FA_ERR_INNER_NULLPTR                                                # last != T
+    st, _, _ = plan(q, k, v, **base, actual_seq_qlen=[5, 5, 12], actual_seq_kvlen=[0, 6, 12])
+    assert st == 0                                                             # empty sequences allowed
+    q4, k4, v4 = qkv((1, 2, 16, 64))
+    assert plan(q4, k4, v4, actual_seq_qlen=[16], actual_seq_kvlen=[16])[0] == fa.FA_ERR_INNER_NULLPTR
+
+
+def test_stats_shapes():
+    q, k, v = qkv((12, 2, 64))
+    base = dict(input_layout="TND", head_num=2, actual_seq_qlen=[12], actual_seq_kvlen=[12])
+    st, _, _ = plan(q, k, v, **base, softmax_max=torch.zeros(12, 2, 8), softmax_sum=torch.zeros(12, 2, 8))
+    assert st == fa.FA_ERR_INNER_NULLPTR   # "" wants [N, T, 8]
+    st, _, _ = plan(q, k, v, **base, softmax_out_layout="same_as_input",
+                    softmax_max=torch.zeros(12, 2, 8), softmax_sum=torch.zeros(12, 2, 8))
+    assert st == 0
+
+
+def test_sink_pse_and_mask_shapes():
+    q, k, v = qkv((2, 2, 16, 64))
+    assert plan(q, k, v, sink=torch.zeros(3))[0] == fa.FA_ERR_INNER_NULLPTR
+    assert plan(q, k, v, sink=torch.zeros(2))[0] == 0
+    assert plan(q, k, v, real_shift=torch.zeros(2, 2, 16, 15, dtype=torch.float16))[0] == fa.FA_ERR_INNER_NULLPTR
+    assert plan(q, k, v, real_shift=torch.zeros(1, 2, 16, 16, dtype=torch.float16))[0] == 0
+    assert plan(q, k, v, real_shift=torch.zeros(3), pse_type=2)[0] == fa.FA_ERR_INNER_NULLPTR
+    assert plan(q, k, v, real_shift=torch.zeros(2, 2), pse_type=2)[0] == 0
+    for shape in [(2, 2, 16, 16), (2, 1, 16, 16), (1, 1, 16, 16), (16, 16)]:
+        assert plan(q, k, v, atten_mask=torch.zeros(shape, dtype=torch.uint8))[0] == 0, shape
+    assert plan(q, k, v, atten_mask=torch.zeros(1, 2, 16, 16, dtype=torch.uint8))[0] == 0
+    for shape in [(16, 15), (3, 1, 16, 16), (2, 3, 16, 16), (16,)]:
+        assert plan(q, k, v, atten_mask=torch.zeros(shape, dtype=torch.bool))[0] == fa.FA_ERR_INNER_NULLPTR, shape

@@ -1,0 +1,275 @@
+"""CUDA path vs the float64 oracle through the C ABI, on the same seeded
+inputs.  Small cases compare every output element and span several 128-row
+tiles with a ragged tail; the five workloads at full size compare sampled rows
+(oracle row by row) in the launch configuration the bench times."""
+import numpy as np
+import pytest
+import torch
+
+import attention_forward_20_b200 as fa
+from workloads import normal, causal_mask_u8, alibi_slopes, cumulative, build, Workload
+from tests.parity import run_gpu, compare_full, compare_rows, sample_rows, f64
+
+pytestmark = pytest.mark.gpu
+INT64_MAX = 2**63 - 1
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    from attention_forward_20_b200 import build as b
+    b.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    yield
+    status, word = fa.device_error()
+    assert status == 0 and word == 0, f"kernel error word {word:#x}"
+
+
+def W(layout, dtype, shape, heads, seed, **kw):
+    """Workload from q/k/v drawn N(0,1) with consecutive seeds."""
+    kshape = kw.pop("kshape", shape)
+    vshape = kw.pop("vshape", kshape)
+    return Workload("case", 0, layout, dtype, heads, normal(shape, dtype, seed), normal(kshape, dtype, seed + 1),
+                    normal(vshape, dtype, seed + 2), scale=kw.pop("scale", None) or
+                    (shape[-1] if layout not in ("BSH", "SBH") else shape[-1] // heads) ** -0.5, **kw)
+
+
+def plan_text(w):
+    q, k, v = w.q.cuda(), w.k.cuda(), w.v.cuda()
+    return fa.plan(q, k, v, input_layout=w.layout, head_num=w.head_num, scale=w.scale,
+                   actual_seq_qlen=w.actual_seq_q, actual_seq_kvlen=w.actual_seq_kv)[2]
+
+
+# ---------------------------------------------------------------------------
+# tcgen05 kernel, dense layouts
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("s", [128, 300, 513])
+def test_dense_bnsd(dtype, d, s):
+    w = W("BNSD", dtype, (2, 3, s, d), 3, 100 + s)
+    assert "sm100_tcgen05" in plan_text(w)
+    compare_full(w)
+
+
+def test_workload_2_shape_reduced():
+    w = build(2, seq_scale=8)   # [2,24,512,128] fp16
+    compare_full(w)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_causal_band_and_sink(dtype):
+    w = W("BSND", dtype, (2, 333, 4, 128), 4, 200, next_tokens=0, sink=normal((4,), "f32", 204))
+    compare_full(w)
+
+
+@pytest.mark.parametrize("mask_mode", [0, 1])
+def test_causal_mask_tensor_with_sink(mask_mode):
+    w = build(3, seq_scale=16)  # [4,512,32,128] bf16, mask [512,512]
+    w.mask_mode = mask_mode
+    compare_full(w)
+
+
+def test_mask_tensor_random_with_band():
+    s = 300
+    w = W("BNSD", "f16", (1, 2, s, 64), 2, 300, pre_tokens=200, next_tokens=40)
+    g = torch.Generator().manual_seed(301)
+    w.atten_mask = (torch.rand(1, 2, s, s, generator=g) < 0.3).to(torch.uint8)
+    compare_full(w)
+
+
+def test_band_alibi_bsh_d64():
+    w = build(5, seq_scale=32)   # [2,512,1024] N=16 D=64, pre=64, next=0, slopes
+    compare_full(w)
+
+
+def test_band_alibi_two_sided():
+    w = W("BNSD", "bf16", (1, 4, 400, 128), 4, 400, pre_tokens=150, next_tokens=70,
+          pse=alibi_slopes(4), pse_type=2)
+    compare_full(w)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_dense_pse_tensor(dtype):
+    s = 260
+    w = W("BNSD", dtype, (2, 2, s, 64), 2, 500, next_tokens=0)
+    w.pse = normal((2, 2, s, s), dtype, 505)
+    w.pse_type = 1
+    compare_full(w)
+    w.pse = normal((1, 2, s, s), dtype, 506)  # broadcast over the batch
+    compare_full(w)
+
+
+def test_sq_differs_from_skv():
+    w = W("BNSD", "f16", (2, 2, 200, 128), 2, 600, kshape=(2, 2, 333, 128))
+    compare_full(w)
+    w = W("BSND", "bf16", (1, 390, 2, 64), 2, 610, kshape=(1, 150, 2, 64), pre_tokens=100, next_tokens=5)
+    compare_full(w)
+
+
+def test_gqa():
+    w = W("BNSD", "bf16", (1, 8, 256, 128), 8, 700, kshape=(1, 2, 256, 128), next_tokens=0)
+    compare_full(w)
+
+
+def test_sbh_layout():
+    w = W("SBH", "f16", (270, 2, 4 * 64), 4, 800, next_tokens=0)
+    compare_full(w)
+
+
+def test_negative_scale():
+    w = W("BNSD", "f16", (1, 2, 200, 64), 2, 900, scale=-0.1)
+    compare_full(w)
+
+
+def test_empty_rows_band_and_sink():
+    # nextTokens = -3: rows 0..2 keep nothing; with a sink they get (0, sink, 1)
+    w = W("BNSD", "bf16", (1, 2, 140, 64), 2, 1000, pre_tokens=10, next_tokens=-3)
+    compare_full(w)
+    w.sink = normal((2,), "f32", 1004)
+    compare_full(w)
+
+
+def test_kv_shorter_than_a_tile_and_single_row():
+    compare_full(W("BNSD", "f16", (1, 1, 1, 128), 1, 1100))
+    compare_full(W("BNSD", "f16", (1, 1, 300, 128), 1, 1110, kshape=(1, 1, 5, 128)))
+
+
+def test_permuted_strides_tma():
+    base = normal((2, 3, 200, 128), "bf16", 1200)
+    w = W("BSND", "bf16", (2, 200, 3, 128), 3, 1210)
+    w.q = base.permute(0, 2, 1, 3)          # BSND view of a BNSD buffer
+    assert not w.q.is_contiguous()
+    compare_full(w)
+
+
+# ---------------------------------------------------------------------------
+# varlen TND
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("stats_layout", ["", "same_as_input"])
+def test_varlen_causal(stats_layout):
+    lens = [300, 0, 129, 1, 513, 64]
+    t = sum(lens)
+    cum = cumulative(lens, leading_zero=False)
+    w = W("TND", "bf16", (t, 3, 128), 3, 1300, next_tokens=0, actual_seq_q=cum, actual_seq_kv=list(cum),
+          softmax_out_layout=stats_layout)
+    compare_full(w)
+
+
+def test_varlen_kv_lengths_differ_with_sink_and_alibi():
+    lq, lk = [100, 260, 0, 7], [300, 10, 5, 129]
+    wq = normal((sum(lq), 2, 64), "f16", 1400)
+    w = W("TND", "f16", (sum(lk), 2, 64), 2, 1401, actual_seq_q=cumulative(lq, False),
+          actual_seq_kv=cumulative(lk, False), pre_tokens=50, next_tokens=20,
+          sink=normal((2,), "f32", 1405), pse=alibi_slopes(2), pse_type=2)
+    w.q = wq
+    compare_full(w)
+
+
+def test_varlen_mask_tensor():
+    lens = [200, 77]
+    cum = cumulative(lens, False)
+    w = W("TND", "bf16", (277, 2, 128), 2, 1500, actual_seq_q=cum, actual_seq_kv=list(cum))
+    w.atten_mask = causal_mask_u8(256, 256)
+    compare_full(w)
+
+
+def test_varlen_workload_4_reduced():
+    compare_full(build(4, seq_scale=4))
+
+
+def test_attention_forward_varlen_api():
+    lens = [128, 300]
+    cu = torch.tensor(cumulative(lens, True), dtype=torch.int32)
+    q, k, v = (normal((428, 2, 128), "bf16", 1600 + i).cuda() for i in range(3))
+    out = fa.attention_forward_varlen(q, k, v, cu, cu, causal=True)
+    w = W("TND", "bf16", (428, 2, 128), 2, 1600, next_tokens=0, actual_seq_q=cumulative(lens, False),
+          actual_seq_kv=cumulative(lens, False))
+    ref_out, _, _ = run_gpu(w)
+    assert torch.equal(out, ref_out)
+
+
+def test_attention_forward_api_layouts():
+    q, k, v = (normal((2, 200, 4, 64), "f16", 1700 + i).cuda() for i in range(3))
+    out_bsnd = fa.attention_forward(q, k, v)
+    out_bnsd = fa.attention_forward(q.transpose(1, 2).contiguous(), k.transpose(1, 2).contiguous(),
+                                    v.transpose(1, 2).contiguous(), head_first=True)
+    assert torch.equal(out_bsnd, out_bnsd.transpose(1, 2))
+
+
+# ---------------------------------------------------------------------------
+# CUDA-core kernel (fp32 and head dims the tensor-core kernel does not take)
+# ---------------------------------------------------------------------------
+
+def test_workload_1_tiny_fp32():
+    w = build(1)
+    assert "simt" in plan_text(w)
+    compare_full(w)
+
+
+@pytest.mark.parametrize("layout", ["BNSD", "BSH", "TND"])
+def test_fp32_features(layout):
+    if layout == "TND":
+        lens = [70, 0, 33]
+        cum = cumulative(lens, False)
+        w = W("TND", "f32", (103, 2, 64), 2, 1800, actual_seq_q=cum, actual_seq_kv=list(cum), next_tokens=0,
+              sink=normal((2,), "f32", 1805), pse=alibi_slopes(2), pse_type=2)
+    elif layout == "BSH":
+        w = W("BSH", "f32", (2, 90, 3 * 32), 3, 1810, pre_tokens=20, next_tokens=3)
+        w.atten_mask = (torch.rand(90, 90, generator=torch.Generator().manual_seed(1811)) < 0.2).to(torch.bool)
+    else:
+        w = W("BNSD", "f32", (1, 2, 77, 96), 2, 1820)
+        w.pse = normal((1, 2, 77, 77), "f32", 1821)
+        w.pse_type = 1
+    compare_full(w)
+
+
+@pytest.mark.parametrize("d", [32, 96, 256])
+def test_half_types_other_head_dims(d):
+    w = W("BNSD", "bf16", (1, 2, 150, d), 2, 1900 + d, next_tokens=0)
+    assert "simt" in plan_text(w)
+    compare_full(w)
+
+
+def test_value_head_dim_smaller():
+    w = W("BNSD", "f16", (1, 2, 100, 128), 2, 2000, vshape=(1, 2, 100, 64))
+    compare_full(w)
+
+
+# ---------------------------------------------------------------------------
+# invariants
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("number", [2, 3])
+def test_deterministic_reruns(number):
+    w = build(number, seq_scale=8)
+    a = run_gpu(w)
+    b = run_gpu(w)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_outputs_fully_written():
+    """NaN-prefilled outputs: every element is overwritten (no gaps)."""
+    w = W("BNSD", "f16", (2, 3, 333, 128), 3, 2100, next_tokens=0)
+    q, k, v = w.q.cuda(), w.k.cuda(), w.v.cuda()
+    out = torch.full_like(q, float("nan"))
+    sm = torch.full((2, 3, 333, 8), float("nan"), device="cuda")
+    ss = torch.full((2, 3, 333, 8), float("nan"), device="cuda")
+    fa.fa_fwd(q, k, v, input_layout="BNSD", head_num=3, next_tokens=0, out=out, softmax_max=sm, softmax_sum=ss)
+    torch.cuda.synchronize()
+    assert not out.isnan().any() and not sm.isnan().any() and not ss.isnan().any()
+
+
+# ---------------------------------------------------------------------------
+# the five workloads at full size, as the bench launches them: sampled rows
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("number", [1, 2, 3, 4, 5])
+def test_full_size_workloads_sampled(number):
+    w = build(number)
+    res = run_gpu(w)
+    for t in res:
+        assert not torch.isnan(t).any()
+    compare_rows(w, res, sample_rows(w, 24, seed=number))
