@@ -21,7 +21,7 @@ FA_MASK_TENSOR, FA_MASK_BAND = 0, 1
 INT64_MAX = 2**63 - 1
 
 EXPORTS = ("fa_fwd_get_workspace_size", "fa_fwd", "fa_executor_destroy",
-           "fa_executor_describe", "fa_device_error", "fa_status_string")
+           "fa_executor_describe", "fa_device_error", "fa_status_string", "fa_fwd_varlen_static")
 
 
 class FaTensor(ctypes.Structure):

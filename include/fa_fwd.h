@@ -160,6 +160,39 @@ FA_API const char* fa_executor_describe(const fa_executor* executor);
  * `detail` is not NULL it receives the raw word (0 when clean). */
 FA_API fa_status fa_device_error(uint64_t* detail);
 
+/* The packed-TND (varlen) forward for callers that cannot allocate device
+ * memory.  The operator pages have no counterpart of this call.
+ *
+ * The ordinary varlen call needs a caller-allocated workspace for its
+ * per-call scratch (cumulative sequence offsets and the work-item table).
+ * Callers that must not call cudaMalloc -- code running while a stream is
+ * captured, or a runtime whose device memory is all handed out up front --
+ * cannot provide one.  This call keeps that scratch in a fixed static device
+ * array of the library instead and allocates nothing: no cudaMalloc/cudaFree,
+ * no workspace, no host heap.  Inputs and outputs are passed as for
+ * fa_fwd_get_workspace_size with inputLayout "TND" (no realShift, no
+ * attenMask, keepProb 1); the work is enqueued on `stream`.
+ *
+ * Limit: nSeq <= 2048 sequences (with T <= 1M tokens, as for every call);
+ * more sequences return FA_ERR_INNER_NULLPTR before any device work.  The
+ * static array (about 130 KB: the offsets and up to 6144 work items) is held
+ * on every GPU that loads the library until the process exits.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call overwrites the part of the array it reads, so nothing
+ * needs clearing, but calls whose work overlaps on the GPU (other streams,
+ * other host threads) race on the shared array.
+ *
+ * Returns FA_SUCCESS, FA_ERR_PARAM_NULLPTR, FA_ERR_PARAM_INVALID,
+ * FA_ERR_INNER_NULLPTR or FA_ERR_CUDA. */
+FA_API fa_status fa_fwd_varlen_static(
+    const fa_tensor* query, const fa_tensor* key, const fa_tensor* value, const fa_tensor* sink,
+    const int64_t* actualSeqQLen, const int64_t* actualSeqKvLen, int64_t nSeq,
+    double scaleValue, int64_t preTokens, int64_t nextTokens, int64_t headNum,
+    const char* softmaxOutLayout, const fa_tensor* softmaxMax, const fa_tensor* softmaxSum,
+    const fa_tensor* attentionOut, void* stream);
+
 /* Human-readable name of a status code (static string). */
 FA_API const char* fa_status_string(fa_status status);
 
