@@ -12,6 +12,11 @@
 //   warps 4-7  softmax tile 1
 //   warp  8    TMA producer     (Q tiles, then K and V 128-row blocks into a ring)
 //   warp  9    MMA issuer       (S = Q·Kᵀ and O += P·V with tcgen05.mma)
+//   warps 10-11 idle (they complete the third warpgroup)
+//
+// The launch gives every thread the same register budget; setmaxnreg then
+// moves registers from the producer/MMA warpgroup (kOtherRegs) to the two
+// softmax warpgroups (kSoftmaxRegs), which hold a whole 128-column S row.
 //
 // TMEM (512 columns): S_t at columns [128t, 128t+128) as fp32; P_t (fp16/bf16,
 // two per column) overwrites the first 64 of them and is the A operand of
@@ -48,7 +53,9 @@ using namespace ptx;
 constexpr int kTileM = 128;     // query rows per tile (one TMEM lane each)
 constexpr int kTileN = 128;     // keys per block
 constexpr int kQBlock = 256;    // query rows per work item (two tiles)
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;   // three warpgroups
+constexpr uint32_t kSoftmaxRegs = 216;  // per thread, softmax warpgroups (setmaxnreg)
+constexpr uint32_t kOtherRegs = 72;     // per thread, producer/MMA warpgroup
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kHeadGroup = 16;  // heads whose items run together, so their K/V stay in L2
@@ -149,7 +156,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
-// TMA producer (one thread)
+// TMA producer (one warp: every lane follows the schedule and waits, so all
+// operands stay warp-uniform; one elected lane issues the copies)
 // ---------------------------------------------------------------------------
 template <int D>
 __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
@@ -178,19 +186,26 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
         const int hi = tr[0].active() ? (tr[1].active() ? max(tr[0].hi, tr[1].hi) : tr[0].hi) : tr[1].hi;
 
         auto load_q = [&](int t) -> bool {
-            if (!mbar_wait(&bars.q_empty[t], (q_fill[t] & 1) ^ 1, abort, kSiteQEmpty)) return false;
-            mbar_arrive_expect_tx(&bars.q_full[t], C::kTileBytes);
-            load_tile(tq, sQ + t * C::kTileBytes, &bars.q_full[t], it.qb * kQBlock + t * kTileM, it.n, it.b,
-                      it.q_off);
+            if (!warp_wait(&bars.q_empty[t], (q_fill[t] & 1) ^ 1, abort, kSiteQEmpty)) return false;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&bars.q_full[t], C::kTileBytes);
+                load_tile(tq, sQ + t * C::kTileBytes, &bars.q_full[t], it.qb * kQBlock + t * kTileM, it.n, it.b,
+                          it.q_off);
+            }
+            __syncwarp();
             ++q_fill[t];
             return true;
         };
         auto load_kv = [&](const CUtensorMap* tm, int jb) -> bool {
             const int slot = kv_fill % C::kStages;
-            if (!mbar_wait(&bars.kv_empty[slot], ((kv_fill / C::kStages) & 1) ^ 1, abort, kSiteKvEmpty))
+            if (!warp_wait(&bars.kv_empty[slot], ((kv_fill / C::kStages) & 1) ^ 1, abort, kSiteKvEmpty))
                 return false;
-            mbar_arrive_expect_tx(&bars.kv_full[slot], C::kTileBytes);
-            load_tile(tm, sKV + slot * C::kTileBytes, &bars.kv_full[slot], jb * kTileN, it.nk, it.b, it.kv_off);
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&bars.kv_full[slot], C::kTileBytes);
+                load_tile(tm, sKV + slot * C::kTileBytes, &bars.kv_full[slot], jb * kTileN, it.nk, it.b,
+                          it.kv_off);
+            }
+            __syncwarp();
             ++kv_fill;
             return true;
         };
@@ -217,7 +232,9 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
 }
 
 // ---------------------------------------------------------------------------
-// MMA issuer (one thread)
+// MMA issuer (one warp, converged: descriptors and TMEM addresses are
+// warp-uniform values; one elected lane issues each tcgen05 instruction, the
+// same lane every time, so its commits cover its MMAs)
 // ---------------------------------------------------------------------------
 template <typename T, int D>
 __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& bars, uint32_t tmem,
@@ -231,31 +248,33 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
 
     auto wait_kv = [&](int* slot) -> bool {
         *slot = kv_use % C::kStages;
-        const bool r = mbar_wait(&bars.kv_full[*slot], (kv_use / C::kStages) & 1, abort, kSiteKvFull);
+        const bool r = warp_wait(&bars.kv_full[*slot], (kv_use / C::kStages) & 1, abort, kSiteKvFull);
         ++kv_use;
         return r;
     };
+    auto commit = [&](uint64_t* bar) {
+        if (elect_one()) tc_commit(bar);
+        __syncwarp();
+    };
     // S_t = Q_t · K^T: D/16 MMAs of K = 16; both operands K-major, 128-byte
     // swizzled, 8-row groups 1024 bytes apart, 64-column chunks one tile-chunk apart.
+    // S_t = Q_t · K^T over D/16 K-steps, O_t (+)= P_t · V over 8 K-steps:
+    // each group is one asm block issued by one elected lane.
     auto issue_qk = [&](int t, int slot) {
-        const uint32_t qa = smem_u32(sQ + t * C::kTileBytes);
-        const uint32_t ka = smem_u32(sKV + slot * C::kTileBytes);
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k >> 2) * C::kChunkBytes + (k & 3) * 32;
-            mma_ss(tmem + t * kTileN, sdesc_sw128(qa + off, 1024, 16), sdesc_sw128(ka + off, 1024, 16), idesc_qk,
-                   k > 0 ? 1u : 0u);
+        const uint64_t qd = sdesc_sw128(smem_u32(sQ + t * C::kTileBytes), 1024, 16);
+        const uint64_t kd = sdesc_sw128(smem_u32(sKV + slot * C::kTileBytes), 1024, 16);
+        if (elect_one()) {
+            if constexpr (D == 128)
+                mma_ss_k128(tmem + t * kTileN, qd, kd, idesc_qk, 0u);
+            else
+                mma_ss_k64(tmem + t * kTileN, qd, kd, idesc_qk, 0u);
         }
+        __syncwarp();
     };
-    // O_t (+)= P_t · V: 8 MMAs of K = 16 keys; P from TMEM (8 columns per step),
-    // V MN-major: 8-key groups 1024 bytes apart, 64-column chunks kChunkBytes apart.
     auto issue_pv = [&](int t, int slot, bool accumulate) {
-        const uint32_t va = smem_u32(sKV + slot * C::kTileBytes);
-#pragma unroll
-        for (int k = 0; k < kTileN / 16; ++k) {
-            mma_ts(tmem + C::kOCol + t * D, tmem + t * kTileN + k * 8, sdesc_sw128(va + k * 2048, 1024, C::kChunkBytes),
-                   idesc_pv, (k > 0 || accumulate) ? 1u : 0u);
-        }
+        const uint64_t vd = sdesc_sw128(smem_u32(sKV + slot * C::kTileBytes), 1024, C::kChunkBytes);
+        if (elect_one()) mma_ts_k128(tmem + C::kOCol + t * D, tmem + t * kTileN, vd, idesc_pv, accumulate ? 1u : 0u);
+        __syncwarp();
     };
 
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
@@ -266,18 +285,18 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
         const int hi = tr[0].active() ? (tr[1].active() ? max(tr[0].hi, tr[1].hi) : tr[0].hi) : tr[1].hi;
 
         for (int t = 0; t < 2; ++t)
-            if (tr[t].active() && !mbar_wait(&bars.q_full[t], q_use[t] & 1, abort, kSiteQFull)) ok = false;
+            if (tr[t].active() && !warp_wait(&bars.q_full[t], q_use[t] & 1, abort, kSiteQFull)) ok = false;
         int sk;
         if (!ok || !wait_kv(&sk)) { ok = false; break; }
         tc_fence_after();
         for (int t = 0; t < 2; ++t) {
             if (tr[t].has(lo)) {
                 issue_qk(t, sk);
-                tc_commit(&bars.s_full[t]);
-                if (lo == tr[t].hi) tc_commit(&bars.q_empty[t]);
+                commit(&bars.s_full[t]);
+                if (lo == tr[t].hi) commit(&bars.q_empty[t]);
             }
         }
-        tc_commit(&bars.kv_empty[sk]);
+        commit(&bars.kv_empty[sk]);
 
         for (int jb = lo; jb <= hi; ++jb) {
             int sv, sk2 = 0;
@@ -286,28 +305,28 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
             tc_fence_after();
             for (int t = 0; t < 2; ++t) {
                 if (tr[t].has(jb)) {
-                    if (!mbar_wait(&bars.p_full[t], p_cnt[t] & 1, abort, kSitePFull)) { ok = false; break; }
+                    if (!warp_wait(&bars.p_full[t], p_cnt[t] & 1, abort, kSitePFull)) { ok = false; break; }
                     ++p_cnt[t];
                     tc_fence_after();
                     issue_pv(t, sv, jb != tr[t].lo);
-                    if (jb == tr[t].hi) tc_commit(&bars.o_full[t]);
+                    if (jb == tr[t].hi) commit(&bars.o_full[t]);
                 }
                 if (has_next && tr[t].has(jb + 1)) {
                     issue_qk(t, sk2);
-                    tc_commit(&bars.s_full[t]);
-                    if (jb + 1 == tr[t].hi) tc_commit(&bars.q_empty[t]);
+                    commit(&bars.s_full[t]);
+                    if (jb + 1 == tr[t].hi) commit(&bars.q_empty[t]);
                 }
             }
             if (!ok) break;
-            tc_commit(&bars.kv_empty[sv]);
-            if (has_next) tc_commit(&bars.kv_empty[sk2]);
+            commit(&bars.kv_empty[sv]);
+            if (has_next) commit(&bars.kv_empty[sk2]);
         }
         for (int t = 0; t < 2; ++t)
             if (tr[t].active()) ++q_use[t];
     }
-    // Drain: every MMA this thread issued completes before TMEM is freed.
-    tc_commit(&bars.drain);
-    mbar_wait(&bars.drain, 0, abort, kSiteDrain);
+    // Drain: every MMA this warp issued completes before TMEM is freed.
+    commit(&bars.drain);
+    warp_wait(&bars.drain, 0, abort, kSiteDrain);
 }
 
 // ---------------------------------------------------------------------------
@@ -316,17 +335,13 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
 __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
+// Two floats rounded to T and packed, `lo` (the lower column) in the low half.
 template <typename T>
-__device__ __forceinline__ uint32_t pack2(float a, float b);
-template <>
-__device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
-    __half2 h = __floats2half2_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&h);
-}
-template <>
-__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&h);
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    if constexpr (std::is_same<T, __nv_bfloat16>::value)
+        return pack_bf16x2(lo, hi);
+    else
+        return pack_f16x2(lo, hi);
 }
 
 // Additive bias of 8 consecutive keys starting at j from a dense pse row (query dtype), times log2(e).
@@ -440,23 +455,45 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, vo
                 }
             }
             {
-                float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+                // columns 0..3 seed four chains; pairs 4..127 feed them in turn
+                float mc[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-                for (int c = 4; c < kTileN; c += 4) {
-                    m0 = fmaxf(m0, s[c]);
-                    m1 = fmaxf(m1, s[c + 1]);
-                    m2 = fmaxf(m2, s[c + 2]);
-                    m3 = fmaxf(m3, s[c + 3]);
-                }
-                m_blk = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+                for (int c = 4; c < kTileN; c += 2) mc[(c >> 1) & 3] = max3(mc[(c >> 1) & 3], s[c], s[c + 1]);
+                m_blk = max3(mc[0], mc[1], fmaxf(mc[2], mc[3]));
                 if constexpr (!kBias) m_blk *= sl2;
             }
 
             const float m_new = fmaxf(m_run, m_blk);
             const bool need = (m_new - m_used) > kRescaleThreshold;  // false while both are -inf
             const float alpha = need ? ex2(m_used - m_new) : 1.f;    // 0 when m_used is -inf
+            if (need) {
+                l *= alpha;
+                m_used = m_new;
+            }
+            m_run = m_new;
+            const float shift = (m_used == -CUDART_INF_F) ? 0.f : m_used;
+
+            // p = 2^(x - shift), two columns per packed FMA / ADD / convert
+            float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+            const float mult = kBias ? 1.f : sl2;
+            const float nshift = -shift;
+            uint32_t pk[64];
+#pragma unroll
+            for (int c = 0; c < kTileN; c += 4) {
+                float x0, x1, x2, x3;
+                fma2(x0, x1, s[c], s[c + 1], mult, mult, nshift, nshift);
+                fma2(x2, x3, s[c + 2], s[c + 3], mult, mult, nshift, nshift);
+                const float e0 = ex2(x0), e1 = ex2(x1), e2 = ex2(x2), e3 = ex2(x3);
+                add2(l0, l1, e0, e1);
+                add2(l2, l3, e2, e3);
+                pk[c / 2] = pack2<T>(e0, e1);
+                pk[c / 2 + 1] = pack2<T>(e2, e3);
+            }
+            l += (l0 + l1) + (l2 + l3);
+            tmem_st_x64(tS, pk);
             if (jb > tr.lo && __any_sync(0xffffffffu, need)) {
-                // O_t is stable: the commit behind this block's S_t covered the last P·V.
+                // Rescale O_t by alpha before this block's P·V is issued.  O_t is
+                // stable: the commit behind this block's S_t covered the last P·V.
 #pragma unroll
                 for (int cc = 0; cc < D; cc += 32) {
                     uint32_t o[32];
@@ -466,38 +503,6 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, vo
                     tmem_st_x32(tO + cc, o);
                 }
             }
-            if (need) {
-                l *= alpha;
-                m_used = m_new;
-            }
-            m_run = m_new;
-            const float shift = (m_used == -CUDART_INF_F) ? 0.f : m_used;
-
-            float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-            uint32_t pk[64];
-#pragma unroll
-            for (int c = 0; c < kTileN; c += 4) {
-                float e0, e1, e2, e3;
-                if constexpr (kBias) {
-                    e0 = ex2(s[c] - shift);
-                    e1 = ex2(s[c + 1] - shift);
-                    e2 = ex2(s[c + 2] - shift);
-                    e3 = ex2(s[c + 3] - shift);
-                } else {
-                    e0 = ex2(fmaf(s[c], sl2, -shift));
-                    e1 = ex2(fmaf(s[c + 1], sl2, -shift));
-                    e2 = ex2(fmaf(s[c + 2], sl2, -shift));
-                    e3 = ex2(fmaf(s[c + 3], sl2, -shift));
-                }
-                l0 += e0;
-                l1 += e1;
-                l2 += e2;
-                l3 += e3;
-                pk[c / 2] = pack2<T>(e0, e1);
-                pk[c / 2 + 1] = pack2<T>(e2, e3);
-            }
-            l += (l0 + l1) + (l2 + l3);
-            tmem_st_x64(tS, pk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars.p_full[t]);
@@ -615,13 +620,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = tmem_base;
 
     if (warp < 8) {
+        setmaxnreg_inc<kSoftmaxRegs>();
         run_softmax<T, D, kBias>(p, bars, tmem, &abort_flag, warp >> 2);
-    } else if (warp == kLoadWarp) {
-        if (lane == 0) run_producer<D>(p, &tmap_q, &tmap_k, &tmap_v, sQ, sKV, bars, &abort_flag);
-        __syncwarp();
     } else {
-        if (lane == 0) run_mma<T, D>(p, sQ, sKV, bars, tmem, &abort_flag);
-        __syncwarp();
+        setmaxnreg_dec<kOtherRegs>();
+        if (warp == kLoadWarp)
+            run_producer<D>(p, &tmap_q, &tmap_k, &tmap_v, sQ, sKV, bars, &abort_flag);
+        else if (warp == kMmaWarp)
+            run_mma<T, D>(p, sQ, sKV, bars, tmem, &abort_flag);
     }
 
     tc_fence_before();
@@ -639,6 +645,14 @@ cudaError_t launch_t(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, co
     auto kern = fa_fwd_sm100_kernel<T, D, kBias>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
+    // setmaxnreg.inc can only hand out what the launch reserved: refuse to
+    // launch (instead of waiting forever) if the compiled register count is
+    // below the split's total.
+    cudaFuncAttributes attr{};
+    e = cudaFuncGetAttributes(&attr, kern);
+    if (e != cudaSuccess) return e;
+    if (static_cast<uint64_t>(attr.numRegs) * kThreads < 2ull * 128 * kSoftmaxRegs + 128ull * kOtherRegs)
+        return cudaErrorLaunchOutOfResources;
     const int grid = p.n_items < num_sms ? p.n_items : num_sms;
     if (grid <= 0) return cudaSuccess;
     kern<<<grid, kThreads, C::kSmemBytes, stream>>>(*reinterpret_cast<const CUtensorMap*>(&tq),

@@ -156,6 +156,84 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         : "memory");
 }
 
+// S (+)= A·B over 4 K-steps of 16: A and B K-major 128-byte-swizzled smem
+// tiles (descriptors for step 0; step k starts (k%4)*32 bytes into 64-column
+// chunk k/4, chunks 16384 bytes apart).  The first step accumulates iff
+// `accumulate`.  One asm block, so nothing is scheduled between the MMAs.
+__device__ __forceinline__ void mma_ss_k64(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .b64 da, db;\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "add.s64 da, %1, 2;\n\tadd.s64 db, %2, 2;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+        "add.s64 da, %1, 4;\n\tadd.s64 db, %2, 4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+        "add.s64 da, %1, 6;\n\tadd.s64 db, %2, 6;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+        "}\n"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// S (+)= A·B over 8 K-steps of 16: A and B K-major 128-byte-swizzled smem
+// tiles (descriptors for step 0; step k starts (k%4)*32 bytes into 64-column
+// chunk k/4, chunks 16384 bytes apart).  The first step accumulates iff
+// `accumulate`.  One asm block, so nothing is scheduled between the MMAs.
+__device__ __forceinline__ void mma_ss_k128(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .b64 da, db;\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "add.s64 da, %1, 2;\n\tadd.s64 db, %2, 2;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+        "add.s64 da, %1, 4;\n\tadd.s64 db, %2, 4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+        "add.s64 da, %1, 6;\n\tadd.s64 db, %2, 6;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+        "add.s64 da, %1, 1024;\n\tadd.s64 db, %2, 1024;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+        "add.s64 da, %1, 1026;\n\tadd.s64 db, %2, 1026;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+        "add.s64 da, %1, 1028;\n\tadd.s64 db, %2, 1028;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+        "add.s64 da, %1, 1030;\n\tadd.s64 db, %2, 1030;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+        "}\n"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// O (+)= P·V over 8 K-steps of 16 keys: P in TMEM (8 columns per step), V an
+// MN-major 128-byte-swizzled smem tile (step k starts k*2048 bytes in).  The
+// first step accumulates iff `accumulate`.
+__device__ __forceinline__ void mma_ts_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .b64 db;\n\t.reg .b32 ta;\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "add.s32 ta, %1, 8;\n\tadd.s64 db, %2, 128;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+        "add.s32 ta, %1, 16;\n\tadd.s64 db, %2, 256;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+        "add.s32 ta, %1, 24;\n\tadd.s64 db, %2, 384;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+        "add.s32 ta, %1, 32;\n\tadd.s64 db, %2, 512;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+        "add.s32 ta, %1, 40;\n\tadd.s64 db, %2, 640;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+        "add.s32 ta, %1, 48;\n\tadd.s64 db, %2, 768;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+        "add.s32 ta, %1, 56;\n\tadd.s64 db, %2, 896;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+        "}\n"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor for a tile written by TMA with 128-byte
 // swizzling: 8-row x 128-byte swizzle atoms, `sbo` bytes between 8-row groups
 // along M/N (K-major) or along K (MN-major), `lbo` bytes between 64-element
@@ -286,6 +364,60 @@ __device__ __forceinline__ void tmem_st_x64(uint32_t taddr, const uint32_t (&r)[
                    "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]),
                    "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
                  : "memory");
+}
+
+// Register budget per thread of the calling warpgroup (all four warps of the
+// warpgroup execute it).  inc waits until the registers are free.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float m;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+    return m;
+}
+
+// (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1) in one packed instruction.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                     float c1) {
+    asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
+        "mov.b64 pa, {%2, %3};\n\t"
+        "mov.b64 pb, {%4, %5};\n\t"
+        "mov.b64 pc, {%6, %7};\n\t"
+        "fma.rn.f32x2 pd, pa, pb, pc;\n\t"
+        "mov.b64 {%0, %1}, pd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// (d0, d1) += (a0, a1) in one packed instruction.
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
+    asm("{\n\t.reg .b64 pa, pd;\n\t"
+        "mov.b64 pa, {%2, %3};\n\t"
+        "mov.b64 pd, {%0, %1};\n\t"
+        "add.rn.f32x2 pd, pd, pa;\n\t"
+        "mov.b64 {%0, %1}, pd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1));
+}
+
+// Two floats rounded (to nearest even) to fp16 / bf16 and packed, `lo` in the
+// low half (the element with the lower column index).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
 }
 
 __device__ __forceinline__ float ex2(float x) {
