@@ -12,6 +12,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <string>
@@ -297,6 +298,9 @@ extern "C" fa_status fa_fwd_get_workspace_size(
     p.has_sink = sink ? 1 : 0;
     p.varlen = L == L_TND ? 1 : 0;
     p.dtype = dt;
+    // Failure injection for tests of the bounded waits (see fa_device_error).
+    const char* stall = std::getenv("FA_DEBUG_STALL");
+    p.debug_stall = (stall && std::atoi(stall) != 0) ? 1 : 0;
 
     p.Tq = (int32_t)qv.S;
     p.Tkv = (int32_t)kv.S;

@@ -56,6 +56,7 @@ struct FaParams {
     int32_t o_vec;              // output rows allow 16-byte stores
     int32_t mask_vec;           // mask rows allow 16-byte loads
     int32_t pse_vec;            // dense bias rows allow 16-byte loads
+    int32_t debug_stall;        // failure injection: the MMA warp waits on a barrier never signalled
 };
 
 enum KernelKind { KERNEL_SIMT = 0, KERNEL_SM100 = 1 };

@@ -66,7 +66,7 @@ constexpr float kRescaleThreshold = 8.0f;
 // wait sites recorded in the error word
 enum : int {
     kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull,
-    kSiteSFull, kSiteOFull, kSiteDrain
+    kSiteSFull, kSiteOFull, kSiteDrain, kSiteInjected
 };
 
 template <int D>
@@ -84,6 +84,7 @@ struct Barriers {
     uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2];
     uint64_t kv_full[8], kv_empty[8];
     uint64_t drain;
+    uint64_t never;  // failure injection: initialised, never arrived on
 };
 
 struct Item {
@@ -245,6 +246,8 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
     constexpr uint32_t idesc_pv = idesc_f16(kBf16, kTileM, D, false, true, false);
     uint32_t kv_use = 0, q_use[2] = {0, 0}, p_cnt[2] = {0, 0};
     bool ok = true;
+    // Failure injection: a wait that can only end by running out of time.
+    if (p.debug_stall && !warp_wait(&bars.never, 0, abort, kSiteInjected)) ok = false;
 
     auto wait_kv = [&](int* slot) -> bool {
         *slot = kv_use % C::kStages;
@@ -602,6 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars.kv_empty[s], 1);
         }
         mbar_init(&bars.drain, 1);
+        mbar_init(&bars.never, 1);
         abort_flag = 0;
         fence_mbar_init();
     }

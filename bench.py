@@ -223,6 +223,30 @@ def time_oracle(w, budget_s, max_heads=None):
     return flops, secs, heads
 
 
+def shard_workload(w, rank):
+    """Rank `rank`'s shard of an N-times larger batch: the workload's shapes,
+    inputs redrawn from a rank-specific seed (rank 0 keeps the workload's own)."""
+    if rank:
+        g = torch.Generator().manual_seed(1000003 * rank)
+        for name in ("q", "k", "v"):
+            t = getattr(w, name)
+            setattr(w, name, torch.randn(t.shape, generator=g, dtype=torch.float32).to(t.dtype))
+    return w
+
+
+def max_over_ranks(values, dist, device):
+    """Element-wise max of a list of floats over all ranks (identity without dist)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def whole_job_tflops(flops_per_rank, world, ms_per_step):
+    """Units all ranks processed per step over the slowest rank's step time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -283,12 +307,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     # each rank: its own shard (seed offset by rank) of the workload's batch
-    w = build(args.workload)
-    if rank:
-        g = torch.Generator().manual_seed(1000003 * rank)
-        for name in ("q", "k", "v"):
-            t = getattr(w, name)
-            setattr(w, name, torch.randn(t.shape, generator=g, dtype=torch.float32).to(t.dtype))
+    w = shard_workload(build(args.workload), rank)
     flops_tiles, flops_exact = tile_flops(w)
     q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
     kw = fa_kwargs(w, dev)
@@ -350,17 +369,14 @@ def main():
     h2d = sum(t.numel() * t.element_size() for t in host)
     d2h = sum(t.numel() * t.element_size() for t in (host_out, host_sm, host_ss))
 
-    t = torch.tensor([kernel_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    kernel_ms, e2e_ms = float(t[0]), float(t[1])
+    kernel_ms, e2e_ms = max_over_ranks([kernel_ms, e2e_ms], dist, dev)
     if dist:
         dist.destroy_process_group()
     if rank != 0:
         return
 
     ms_per_step = kernel_ms / args.steps
-    value = flops_tiles * world / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(flops_tiles, world, ms_per_step)
     per_gpu = flops_tiles / (ms_per_step * 1e-3) / 1e12
     peak, peak_src = load_peak()
     traffic = load_traffic(w.name)
@@ -379,7 +395,7 @@ def main():
         "cpu_baseline": {"value": cpu_value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                          "sample": f"{heads} whole (batch, head) pairs of the workload, float64 NumPy, "
                                    f"{secs:.1f} s"},
-        "e2e": {"value": flops_tiles * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        "e2e": {"value": whole_job_tflops(flops_tiles, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),

@@ -154,10 +154,14 @@ FA_API void fa_executor_destroy(fa_executor* executor);
 FA_API const char* fa_executor_describe(const fa_executor* executor);
 
 /* Reads and clears the current device's kernel error word.  Every wait in the
- * tcgen05 kernel has a time limit; a wait that runs out records an error
- * here and the kernel returns early instead of hanging.  Synchronises the
- * device.  Returns FA_SUCCESS, FA_ERR_DEVICE_TIMEOUT or FA_ERR_CUDA; when
- * `detail` is not NULL it receives the raw word (0 when clean). */
+ * tcgen05 kernel has a time limit (about 2 s); a wait that runs out records an
+ * error here and the kernel returns early instead of hanging.  The raw word
+ * holds the wait site in its high 32 bits and 1 + the CTA index in its low 32
+ * bits.  Synchronises the device.  Returns FA_SUCCESS, FA_ERR_DEVICE_TIMEOUT or
+ * FA_ERR_CUDA; when `detail` is not NULL it receives the raw word (0 when
+ * clean).  For tests of this path, the environment variable FA_DEBUG_STALL=1
+ * (read by fa_fwd_get_workspace_size) makes the kernel wait on a barrier that
+ * is never signalled. */
 FA_API fa_status fa_device_error(uint64_t* detail);
 
 /* The packed-TND (varlen) forward for callers that cannot allocate device

@@ -1,0 +1,39 @@
+"""Failure detection on the GPU without a GPU fault: every wait of the tcgen05
+kernel is bounded.  FA_DEBUG_STALL=1 makes the kernel wait on a barrier that
+is never signalled; the wait runs out after about two seconds, the kernel
+winds down (drains its copies and MMAs, frees TMEM, returns), the host reads
+FA_ERR_DEVICE_TIMEOUT from the error word, and the context stays usable."""
+import pytest
+import torch
+
+import attention_forward_20_b200 as fa
+from tests.parity import compare_full
+from workloads import Workload, normal
+
+pytestmark = pytest.mark.gpu
+
+KNOWN_SITES = set(range(1, 10))
+
+
+def small():
+    shape = (1, 2, 300, 128)
+    return Workload("stall", 0, "BNSD", "bf16", 2, normal(shape, "bf16", 61), normal(shape, "bf16", 62),
+                    normal(shape, "bf16", 63), scale=128 ** -0.5, next_tokens=0)
+
+
+def test_stalled_wait_reports_timeout_and_context_survives(monkeypatch):
+    from attention_forward_20_b200 import build
+    build.build()
+    fa.device_error()  # start clean
+    w = small()
+    monkeypatch.setenv("FA_DEBUG_STALL", "1")
+    q, k, v = w.q.cuda(), w.k.cuda(), w.v.cuda()
+    fa.fa_fwd(q, k, v, input_layout="BNSD", head_num=2, next_tokens=0)
+    status, word = fa.device_error()  # synchronises
+    assert status == fa.FA_ERR_DEVICE_TIMEOUT
+    assert (word >> 32) in KNOWN_SITES and 1 <= (word & 0xFFFFFFFF) <= 148
+    monkeypatch.delenv("FA_DEBUG_STALL")
+    # the context is intact: the next call is correct and clean
+    compare_full(w)
+    assert fa.device_error() == (fa.FA_SUCCESS, 0)
+    torch.cuda.synchronize()
