@@ -25,6 +25,7 @@ struct fa_executor {
     std::vector<int4> table;   // TND, tcgen05 kernel: one entry per (sequence, query block)
     uint64_t off_cu = 0;
     uint64_t off_table = 0;
+    uint64_t off_part = 0;
     uint64_t ws_bytes = 0;
     std::string desc;
 };
@@ -39,6 +40,8 @@ constexpr int64_t kMaxS = 1 << 20;     // S, T 1~1M
 constexpr int64_t kMaxD = 256;         // this library: head dim up to 256
 constexpr int kQBlock = 256;           // tcgen05 kernel: two 128-row query tiles per work item
 constexpr int kKvBlock = 128;
+constexpr uint64_t kScheduleHeader = 256; // tcgen05 kernel: ticket counter at workspace offset 0
+constexpr int kDefaultSms = 148;          // B200
 
 bool parse_layout(const char* s, Layout* out) {
     if (s == nullptr) return false;
@@ -97,6 +100,17 @@ int64_t clamp64(int64_t x, int64_t lo, int64_t hi) { return x < lo ? lo : (x > h
 
 // Number of 128-key blocks that 128-row query tile [r0, r0+128) touches,
 // for the LPT ordering of the varlen work table.
+// 128-key blocks of the union of the two tiles' key ranges of the query block
+// starting at row r0 (0 when neither tile has a key).
+int64_t union_blocks(int64_t r0, int64_t q_len, int64_t kv_len, int64_t pre, int64_t next) {
+    const int64_t r1 = std::min(q_len, r0 + 256) - 1;
+    if (r1 < r0 || kv_len <= 0) return 0;
+    const int64_t lo = std::max<int64_t>(0, r0 - pre);
+    const int64_t hi = std::min<int64_t>(kv_len - 1, r1 + next);
+    if (hi < lo) return 0;
+    return hi / kKvBlock - lo / kKvBlock + 1;
+}
+
 int64_t kv_blocks_for_tile(int64_t r0, int64_t q_len, int64_t kv_len, int64_t pre, int64_t next) {
     const int64_t r1 = std::min(q_len, r0 + 128) - 1;
     if (r1 < r0 || kv_len <= 0) return 0;
@@ -328,8 +342,10 @@ extern "C" fa_status fa_fwd_get_workspace_size(
     const bool sm100 = (dt == FA_F16 || dt == FA_BF16) && qv.D == vv.D && (qv.D == 64 || qv.D == 128) && tma_ok;
     ex->kind = sm100 ? fa::KERNEL_SM100 : fa::KERNEL_SIMT;
 
-    // ---- workspace: cumulative lengths and the varlen work table ----------
+    // ---- workspace: schedule counter, cumulative lengths, varlen work
+    // table, partial results of split items ----------------------------------
     uint64_t off = 0;
+    if (sm100) off = kScheduleHeader;  // the ticket counter, zeroed before every launch
     if (L == L_TND) {
         ex->off_cu = off;
         off += ex->cu.size() * sizeof(int64_t);
@@ -360,15 +376,46 @@ extern "C" fa_status fa_fwd_get_workspace_size(
             p.items_per_n_block = (int32_t)(B * qv.N);
             p.n_items = p.n_qb * p.items_per_n_block;
         }
+        // Equal-cost items (every query block touches the same number of key
+        // blocks) may have their last wave split into key pieces.
+        bool uniform = L != L_TND;
+        int64_t item_blocks = 0;
+        if (uniform) {
+            auto cost = [&](int64_t r0) {
+                return kv_blocks_for_tile(r0, max_q, max_kv, pre_c, next_c) +
+                       kv_blocks_for_tile(r0 + 128, max_q, max_kv, pre_c, next_c);
+            };
+            item_blocks = union_blocks(0, max_q, max_kv, pre_c, next_c);
+            const int64_t c0 = cost(0);
+            for (int64_t qb = 1; uniform && qb < p.n_qb; ++qb)
+                uniform = cost(qb * kQBlock) == c0 && union_blocks(qb * kQBlock, max_q, max_kv, pre_c, next_c) == item_blocks;
+        }
+        // SM count of the current device (an attribute query, no device work);
+        // without a device the plan assumes a full B200.  Any grid is correct:
+        // the SM count only shapes the schedule.
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+            (void)cudaGetLastError();
+            sms = kDefaultSms;
+        }
+        const uint64_t part_bytes = fa::plan_sm100_schedule(p, sms, uniform, (int)item_blocks);
+        if (part_bytes) {
+            off = (off + 255) & ~uint64_t(255);
+            ex->off_part = off;
+            off += part_bytes;
+        }
     }
     ex->ws_bytes = off;
     *workspaceSize = off;
 
     char buf[256];
-    std::snprintf(buf, sizeof(buf), "kernel=%s dtype=%s D=%d Dv=%d B=%d Nq=%d Nkv=%d Sq=%d Skv=%d varlen=%d items=%d ws=%llu",
+    std::snprintf(buf, sizeof(buf),
+                  "kernel=%s dtype=%s D=%d Dv=%d B=%d Nq=%d Nkv=%d Sq=%d Skv=%d varlen=%d items=%d grid=%d "
+                  "dynamic=%d split_items=%d pieces=%d ws=%llu",
                   sm100 ? "sm100_tcgen05" : "simt_fp32acc", dt == FA_F32 ? "f32" : dt == FA_F16 ? "f16" : "bf16",
-                  p.D, p.Dv, p.B, p.Nq, p.Nkv, p.Sq, p.Skv, p.varlen, p.n_items,
-                  (unsigned long long)off);
+                  p.D, p.Dv, p.B, p.Nq, p.Nkv, p.Sq, p.Skv, p.varlen, p.n_items, p.grid,
+                  p.dynamic, p.n_items - p.n_whole, p.n_pieces, (unsigned long long)off);
     ex->desc = buf;
     (void)innerPrecise;
     *executor = ex;
@@ -401,13 +448,12 @@ extern "C" fa_status fa_fwd(void* workspace, uint64_t workspaceSize, fa_executor
     }
     cudaError_t err;
     if (ex->kind == fa::KERNEL_SM100) {
-        int dev = 0, sms = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return done(FA_ERR_CUDA);
+        p.sched_counter = reinterpret_cast<int*>(ws);
+        p.part = ex->off_part ? reinterpret_cast<float*>(ws + ex->off_part) : nullptr;
+        if (p.grid > 0 && p.dynamic && cudaMemsetAsync(ws, 0, sizeof(int), st) != cudaSuccess) return done(FA_ERR_CUDA);
         fa::TmaDesc tq, tk, tv;
         if (fa::make_sm100_tmaps(p, &tq, &tk, &tv) != cudaSuccess) return done(FA_ERR_CUDA);
-        err = fa::launch_sm100(p, tq, tk, tv, sms, st);
+        err = fa::launch_sm100(p, tq, tk, tv, p.grid, st);
     } else {
         err = fa::launch_simt(p, st);
     }

@@ -57,7 +57,23 @@ struct FaParams {
     int32_t mask_vec;           // mask rows allow 16-byte loads
     int32_t pse_vec;            // dense bias rows allow 16-byte loads
     int32_t debug_stall;        // failure injection: the MMA warp waits on a barrier never signalled
+
+    // Schedule: tickets [0, n_whole) are whole work items; ticket
+    // n_whole + u*n_pieces + j is piece j (a contiguous share of the key
+    // blocks) of work item n_whole + u.  CTAs take tickets round-robin, or,
+    // when items differ in cost, the next one from an atomic counter.
+    int* sched_counter;         // device, zero at launch
+    int32_t n_tickets;
+    int32_t n_whole;
+    int32_t n_pieces;           // 0 when no item is split
+    int32_t grid;               // CTAs of the tcgen05 kernel
+    int32_t dynamic;            // 1: tickets from sched_counter; 0: round-robin
+    float* part;                // split items: [item u][piece j][256 rows][D + 4] fp32:
+                                // O relative to m_used, then m_run, m_used, l (log2 units)
 };
+
+// fp32 words per row of a partial result
+inline int part_row_words(int d) { return d + 4; }
 
 enum KernelKind { KERNEL_SIMT = 0, KERNEL_SM100 = 1 };
 
@@ -69,6 +85,12 @@ struct alignas(64) TmaDesc {
 cudaError_t launch_simt(const FaParams& p, cudaStream_t stream);
 cudaError_t launch_sm100(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk,
                          const TmaDesc& tv, int num_sms, cudaStream_t stream);
+// Schedule of the tcgen05 kernel (fills grid, n_whole, n_pieces, n_tickets
+// from n_items): one CTA per SM, and, when every work item costs the same
+// (`uniform`, item_kv_blocks 128-key blocks each) and the last wave is short,
+// the last wave's items split into key pieces.  Returns the bytes of partial
+// results the split needs (0 without a split).
+uint64_t plan_sm100_schedule(FaParams& p, int num_sms, bool uniform, int item_kv_blocks);
 // Encodes the Q/K/V tensor maps for the tcgen05 kernel.
 cudaError_t make_sm100_tmaps(const FaParams& p, TmaDesc* tq, TmaDesc* tk, TmaDesc* tv);
 uint64_t read_and_clear_device_error(cudaError_t* err);

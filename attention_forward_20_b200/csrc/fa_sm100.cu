@@ -62,11 +62,16 @@ constexpr int kHeadGroup = 16;  // heads whose items run together, so their K/V 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kSched = 4;            // ticket slots between the TMA warp and the other warps
+constexpr int kTicketEnd = -1;       // no work left
+constexpr int kTicketAbort = -2;     // a bounded wait gave up
+constexpr int kTicketReaders = 9;    // the MMA warp and the eight softmax warps
+constexpr int kMergeThreads = 256;
 
 // wait sites recorded in the error word
 enum : int {
     kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull,
-    kSiteSFull, kSiteOFull, kSiteDrain, kSiteInjected
+    kSiteSFull, kSiteOFull, kSiteDrain, kSiteInjected, kSiteSched
 };
 
 template <int D>
@@ -83,8 +88,10 @@ struct Cfg {
 struct Barriers {
     uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2];
     uint64_t kv_full[8], kv_empty[8];
+    uint64_t sched_full[kSched], sched_empty[kSched];
     uint64_t drain;
     uint64_t never;  // failure injection: initialised, never arrived on
+    int ticket[kSched];
 };
 
 struct Item {
@@ -151,9 +158,87 @@ __device__ __forceinline__ TileRange tile_range(const FaParams& p, const Item& i
     return r;
 }
 
+// What a ticket stands for: a whole work item, or piece `piece` of split
+// item number `tail` (counted among the split ones), whose tiles then only
+// cover that piece's share of the item's key blocks.
+struct Work {
+    Item it;
+    TileRange tr[2];
+    int piece;  // -1: the whole item
+    int tail;
+};
+
+__device__ __forceinline__ Work work_of(const FaParams& p, int ticket) {
+    Work w;
+    int item = ticket;
+    w.piece = -1;
+    w.tail = 0;
+    if (ticket >= p.n_whole) {
+        const int u = ticket - p.n_whole;
+        w.tail = u / p.n_pieces;
+        w.piece = u - w.tail * p.n_pieces;
+        item = p.n_whole + w.tail;
+    }
+    w.it = decode_item(p, item);
+    w.tr[0] = tile_range(p, w.it, 0);
+    w.tr[1] = tile_range(p, w.it, 1);
+    if (w.piece >= 0 && (w.tr[0].active() || w.tr[1].active())) {
+        const int lo = w.tr[0].active() ? (w.tr[1].active() ? min(w.tr[0].lo, w.tr[1].lo) : w.tr[0].lo) : w.tr[1].lo;
+        const int hi = w.tr[0].active() ? (w.tr[1].active() ? max(w.tr[0].hi, w.tr[1].hi) : w.tr[0].hi) : w.tr[1].hi;
+        const int n = hi - lo + 1;
+        const int c0 = lo + (w.piece * n) / p.n_pieces;
+        const int c1 = lo + ((w.piece + 1) * n) / p.n_pieces - 1;
+        for (int t = 0; t < 2; ++t) {
+            if (w.tr[t].active()) {
+                w.tr[t].lo = max(w.tr[t].lo, c0);
+                w.tr[t].hi = min(w.tr[t].hi, c1);
+                if (w.tr[t].hi < w.tr[t].lo) {  // no block of this tile in the piece
+                    w.tr[t].lo = 0;
+                    w.tr[t].hi = -1;
+                }
+            }
+        }
+    }
+    return w;
+}
+
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int site) {
     const bool ok = mbar_wait(bar, parity, abort, site);
     return __all_sync(0xffffffffu, ok);
+}
+
+// Tickets.  Equal-cost items (p.dynamic == 0) go round-robin: the k-th ticket
+// of CTA c is c + k * gridDim.x, which every warp computes for itself.
+// Otherwise the TMA warp takes the next ticket from the global counter as soon
+// as it has issued the loads of the previous one, and hands it to the MMA warp
+// and the softmax warps through kSched shared-memory slots.
+__device__ __forceinline__ int static_ticket(const FaParams& p, uint32_t& k) {
+    const int tk = blockIdx.x + static_cast<int>(k++) * gridDim.x;
+    return tk < p.n_tickets ? tk : kTicketEnd;
+}
+__device__ __forceinline__ int take_ticket_global(const FaParams& p, Barriers& bars, uint32_t& k, volatile int* abort) {
+    if (!p.dynamic) return static_ticket(p, k);
+    const uint32_t slot = k % kSched;
+    if (!warp_wait(&bars.sched_empty[slot], ((k / kSched) & 1) ^ 1, abort, kSiteSched)) return kTicketAbort;
+    int tk = 0;
+    if ((threadIdx.x & 31) == 0) {
+        tk = atomicAdd(p.sched_counter, 1);
+        if (tk >= p.n_tickets) tk = kTicketEnd;
+        bars.ticket[slot] = tk;
+        mbar_arrive(&bars.sched_full[slot]);
+    }
+    ++k;
+    return __shfl_sync(0xffffffffu, tk, 0);
+}
+__device__ __forceinline__ int take_ticket_local(const FaParams& p, Barriers& bars, uint32_t& k, volatile int* abort) {
+    if (!p.dynamic) return static_ticket(p, k);
+    const uint32_t slot = k % kSched;
+    if (!warp_wait(&bars.sched_full[slot], (k / kSched) & 1, abort, kSiteSched)) return kTicketAbort;
+    const int tk = *reinterpret_cast<volatile int*>(&bars.ticket[slot]);
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&bars.sched_empty[slot]);
+    ++k;
+    return tk;
 }
 
 // ---------------------------------------------------------------------------
@@ -165,7 +250,7 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
                              const CUtensorMap* tv, uint8_t* sQ, uint8_t* sKV, Barriers& bars,
                              volatile int* abort) {
     using C = Cfg<D>;
-    uint32_t kv_fill = 0, q_fill[2] = {0, 0};
+    uint32_t kv_fill = 0, q_fill[2] = {0, 0}, k_sched = 0;
     bool ok = true;
 
     auto load_tile = [&](const CUtensorMap* tm, uint8_t* dst, uint64_t* bar, int row, int head, int b,
@@ -179,9 +264,13 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
         }
     };
 
-    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const Item it = decode_item(p, item);
-        const TileRange tr[2] = {tile_range(p, it, 0), tile_range(p, it, 1)};
+    while (ok) {
+        const int ticket = take_ticket_global(p, bars, k_sched, abort);
+        if (ticket == kTicketAbort) { ok = false; break; }
+        if (ticket == kTicketEnd) break;
+        const Work wk = work_of(p, ticket);
+        const Item& it = wk.it;
+        const TileRange* tr = wk.tr;
         if (!tr[0].active() && !tr[1].active()) continue;
         const int lo = tr[0].active() ? (tr[1].active() ? min(tr[0].lo, tr[1].lo) : tr[0].lo) : tr[1].lo;
         const int hi = tr[0].active() ? (tr[1].active() ? max(tr[0].hi, tr[1].hi) : tr[0].hi) : tr[1].hi;
@@ -244,7 +333,7 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     const uint32_t idesc_qk = idesc_f16(kBf16, kTileM, kTileN, false, false, p.neg_scale != 0);
     constexpr uint32_t idesc_pv = idesc_f16(kBf16, kTileM, D, false, true, false);
-    uint32_t kv_use = 0, q_use[2] = {0, 0}, p_cnt[2] = {0, 0};
+    uint32_t kv_use = 0, q_use[2] = {0, 0}, p_cnt[2] = {0, 0}, k_sched = 0;
     bool ok = true;
     // Failure injection: a wait that can only end by running out of time.
     if (p.debug_stall && !warp_wait(&bars.never, 0, abort, kSiteInjected)) ok = false;
@@ -280,9 +369,12 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
         __syncwarp();
     };
 
-    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const Item it = decode_item(p, item);
-        const TileRange tr[2] = {tile_range(p, it, 0), tile_range(p, it, 1)};
+    while (ok) {
+        const int ticket = take_ticket_local(p, bars, k_sched, abort);
+        if (ticket == kTicketAbort) { ok = false; break; }
+        if (ticket == kTicketEnd) break;
+        const Work wk = work_of(p, ticket);
+        const TileRange* tr = wk.tr;
         if (!tr[0].active() && !tr[1].active()) continue;
         const int lo = tr[0].active() ? (tr[1].active() ? min(tr[0].lo, tr[1].lo) : tr[0].lo) : tr[1].lo;
         const int hi = tr[0].active() ? (tr[1].active() ? max(tr[0].hi, tr[1].hi) : tr[0].hi) : tr[1].hi;
@@ -377,6 +469,63 @@ __device__ __forceinline__ uint32_t load_mask16(const uint8_t* row, int j, int c
     return bits;
 }
 
+// Final statistics of a row from its running max m_run, the max m_used that
+// O and l are relative to, and l (all log2 units): the sink joins the max and
+// the denominator; o_scale turns O into the output.
+struct RowFinal {
+    float m_f, l_f, o_scale;
+};
+__device__ __forceinline__ RowFinal finalize_row(const FaParams& p, const Item& it, float m_run, float m_used, float l) {
+    RowFinal f;
+    f.m_f = m_run;
+    if (p.has_sink) {
+        const float sk = p.sink[it.n] * kLog2e;
+        f.m_f = fmaxf(m_run, sk);
+        const float a = (m_used == -CUDART_INF_F) ? 0.f : ex2(m_used - f.m_f);
+        f.l_f = l * a + ex2(sk - f.m_f);
+        f.o_scale = a / f.l_f;
+    } else {
+        f.l_f = l * ((m_used == -CUDART_INF_F) ? 0.f : ex2(m_used - m_run));
+        f.o_scale = (l > 0.f) ? 1.f / l : 0.f;
+    }
+    return f;
+}
+
+// 32 output columns of a row (fp32 bits in o) scaled, rounded to T and stored.
+template <typename T>
+__device__ __forceinline__ void store_out32(const FaParams& p, T* orow, int cc, const uint32_t (&o)[32], float o_scale) {
+    uint32_t w[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+        w[e] = pack2<T>(__uint_as_float(o[2 * e]) * o_scale, __uint_as_float(o[2 * e + 1]) * o_scale);
+    if (p.o_vec) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + cc);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+    } else {
+        uint32_t* dst = reinterpret_cast<uint32_t*>(orow + cc);
+        if ((reinterpret_cast<uintptr_t>(dst) & 3u) == 0) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) dst[e] = w[e];
+        } else {
+            const T* h = reinterpret_cast<const T*>(w);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orow[cc + e] = h[e];
+        }
+    }
+}
+
+// softmaxMax (natural log units) and softmaxSum of query row i, all 8 lanes.
+__device__ __forceinline__ void store_stats(const FaParams& p, const Item& it, int i, const RowFinal& f) {
+    const int64_t so = it.b * p.st_b + it.n * p.st_n + (it.q_off + i) * p.st_s;
+    const float m_nat = f.m_f * kLn2;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        p.smax[so + e] = m_nat;
+        p.ssum[so + e] = f.l_f;
+    }
+}
+
 template <typename T, int D, bool kBias>
 __device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, volatile int* abort, int t) {
     using C = Cfg<D>;
@@ -386,12 +535,16 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, vo
     const uint32_t tS = tmem + lane_off + t * kTileN;
     const uint32_t tO = tmem + lane_off + C::kOCol + t * D;
     const float sl2 = p.scale_log2;
-    uint32_t s_cnt = 0, o_cnt = 0;
+    uint32_t s_cnt = 0, o_cnt = 0, k_sched = 0;
     bool ok = true;
 
-    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const Item it = decode_item(p, item);
-        const TileRange tr = tile_range(p, it, t);
+    while (ok) {
+        const int ticket = take_ticket_local(p, bars, k_sched, abort);
+        if (ticket == kTicketAbort) { ok = false; break; }
+        if (ticket == kTicketEnd) break;
+        const Work wk = work_of(p, ticket);
+        const Item& it = wk.it;
+        const TileRange tr = wk.tr[t];
         if (!tr.valid) continue;
         const int r0 = it.qb * kQBlock + t * kTileM;
         const int i = r0 + row;
@@ -519,18 +672,30 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, vo
             ++o_cnt;
             tc_fence_after();
         }
-        float m_f = m_run, l_f, o_scale;
-        if (p.has_sink) {
-            const float sk = p.sink[it.n] * kLog2e;
-            m_f = fmaxf(m_run, sk);
-            const float a = (m_used == -CUDART_INF_F) ? 0.f : ex2(m_used - m_f);
-            l_f = l * a + ex2(sk - m_f);
-            o_scale = a / l_f;
-        } else {
-            l_f = l * ((m_used == -CUDART_INF_F) ? 0.f : ex2(m_used - m_run));
-            o_scale = (l > 0.f) ? 1.f / l : 0.f;
+        if (wk.piece >= 0) {
+            // A piece of a split item: keep O_t (relative to m_used) and the
+            // row's m_run, m_used, l for the merge.
+            float* prow = p.part + ((static_cast<size_t>(wk.tail) * p.n_pieces + wk.piece) * kQBlock + t * kTileM + row) *
+                                       static_cast<size_t>(D + 4);
+#pragma unroll
+            for (int cc = 0; cc < D; cc += 32) {
+                uint32_t o[32];
+                if (has_blocks) {
+                    tmem_ld_x32(tO + cc, o);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = 0u;
+                }
+                float4* dst = reinterpret_cast<float4*>(prow + cc);
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                    dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                         __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+            }
+            *reinterpret_cast<float4*>(prow + D) = make_float4(m_run, m_used, l, 0.f);
+            continue;
         }
-
+        const RowFinal f = finalize_row(p, it, m_run, m_used, l);
         T* orow = static_cast<T*>(p.o) + it.b * p.o_b + it.n * p.o_n + (it.q_off + i) * p.o_s;
 #pragma unroll
         for (int cc = 0; cc < D; cc += 32) {
@@ -541,38 +706,74 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, vo
 #pragma unroll
                 for (int e = 0; e < 32; ++e) o[e] = 0u;
             }
-            uint32_t w[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                w[e] = pack2<T>(__uint_as_float(o[2 * e]) * o_scale, __uint_as_float(o[2 * e + 1]) * o_scale);
-            if (row_ok) {
-                if (p.o_vec) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + cc);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-                } else {
-                    uint32_t* dst = reinterpret_cast<uint32_t*>(orow + cc);
-                    if ((reinterpret_cast<uintptr_t>(dst) & 3u) == 0) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) dst[e] = w[e];
-                    } else {
-                        const T* h = reinterpret_cast<const T*>(w);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) orow[cc + e] = h[e];
-                    }
-                }
-            }
+            if (row_ok) store_out32<T>(p, orow, cc, o, f.o_scale);
         }
-        if (row_ok) {
-            const int64_t so = it.b * p.st_b + it.n * p.st_n + (it.q_off + i) * p.st_s;
-            const float m_nat = m_f * kLn2;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                p.smax[so + e] = m_nat;
-                p.ssum[so + e] = l_f;
-            }
+        if (row_ok) store_stats(p, it, i, f);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Merge of split items: the online-softmax combination of the pieces' partial
+// results (applied to whole pieces instead of key blocks), then the same row
+// finish as the softmax epilogue.  One thread per (query row, 8 output
+// columns): a warp reads two rows' partials in 32-byte runs.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(kMergeThreads) fa_merge_kernel(const FaParams p) {
+    constexpr int kGroups = D / 8;
+    const int n_split = (p.n_tickets - p.n_whole) / p.n_pieces;
+    const int idx = blockIdx.x * kMergeThreads + threadIdx.x;
+    if (idx >= n_split * kQBlock * kGroups) return;
+    const int g = idx % kGroups;
+    const int rr = idx / kGroups;
+    const int r = rr % kQBlock, u = rr / kQBlock;
+    const Item it = decode_item(p, p.n_whole + u);
+    const int i = it.qb * kQBlock + r;
+    if (i >= it.q_len) return;
+    const size_t words = D + 4;
+    const float* base = p.part + (static_cast<size_t>(u) * p.n_pieces * kQBlock + r) * words;
+    const size_t piece_stride = static_cast<size_t>(kQBlock) * words;
+    float m_run = -CUDART_INF_F, m_used = -CUDART_INF_F;
+    for (int j = 0; j < p.n_pieces; ++j) {
+        const float4 st = *reinterpret_cast<const float4*>(base + j * piece_stride + D);
+        m_run = fmaxf(m_run, st.x);
+        m_used = fmaxf(m_used, st.y);
+    }
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float l = 0.f;
+    if (m_used != -CUDART_INF_F) {
+#pragma unroll 4
+        for (int j = 0; j < p.n_pieces; ++j) {
+            const float* pr = base + j * piece_stride;
+            const float4 st = *reinterpret_cast<const float4*>(pr + D);
+            const float4 o0 = *reinterpret_cast<const float4*>(pr + 8 * g);
+            const float4 o1 = *reinterpret_cast<const float4*>(pr + 8 * g + 4);
+            // a piece that saw no key of this row has m_used = -inf: weight 0
+            const float w = (st.y == -CUDART_INF_F) ? 0.f : ex2(st.y - m_used);
+            l = fmaf(st.z, w, l);
+            acc[0] = fmaf(o0.x, w, acc[0]);
+            acc[1] = fmaf(o0.y, w, acc[1]);
+            acc[2] = fmaf(o0.z, w, acc[2]);
+            acc[3] = fmaf(o0.w, w, acc[3]);
+            acc[4] = fmaf(o1.x, w, acc[4]);
+            acc[5] = fmaf(o1.y, w, acc[5]);
+            acc[6] = fmaf(o1.z, w, acc[6]);
+            acc[7] = fmaf(o1.w, w, acc[7]);
         }
     }
+    const RowFinal f = finalize_row(p, it, m_run, m_used, l);
+    T* orow = static_cast<T*>(p.o) + it.b * p.o_b + it.n * p.o_n + (it.q_off + i) * p.o_s + 8 * g;
+    uint32_t w4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w4[e] = pack2<T>(acc[2 * e] * f.o_scale, acc[2 * e + 1] * f.o_scale);
+    if (p.o_vec) {
+        *reinterpret_cast<uint4*>(orow) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    } else {
+        const T* h = reinterpret_cast<const T*>(w4);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) orow[e] = h[e];
+    }
+    if (g == 0) store_stats(p, it, i, f);
 }
 
 // ---------------------------------------------------------------------------
@@ -603,6 +804,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&bars.kv_full[s], 1);
             mbar_init(&bars.kv_empty[s], 1);
+        }
+        for (int k = 0; k < kSched; ++k) {
+            mbar_init(&bars.sched_full[k], 1);
+            mbar_init(&bars.sched_empty[k], kTicketReaders);
         }
         mbar_init(&bars.drain, 1);
         mbar_init(&bars.never, 1);
@@ -657,11 +862,16 @@ cudaError_t launch_t(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, co
     if (e != cudaSuccess) return e;
     if (static_cast<uint64_t>(attr.numRegs) * kThreads < 2ull * 128 * kSoftmaxRegs + 128ull * kOtherRegs)
         return cudaErrorLaunchOutOfResources;
-    const int grid = p.n_items < num_sms ? p.n_items : num_sms;
-    if (grid <= 0) return cudaSuccess;
-    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(*reinterpret_cast<const CUtensorMap*>(&tq),
-                                                    *reinterpret_cast<const CUtensorMap*>(&tk),
-                                                    *reinterpret_cast<const CUtensorMap*>(&tv), p);
+    (void)num_sms;
+    if (p.grid <= 0) return cudaSuccess;
+    kern<<<p.grid, kThreads, C::kSmemBytes, stream>>>(*reinterpret_cast<const CUtensorMap*>(&tq),
+                                                      *reinterpret_cast<const CUtensorMap*>(&tk),
+                                                      *reinterpret_cast<const CUtensorMap*>(&tv), p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.n_pieces == 0) return e;
+    const int n_split = (p.n_tickets - p.n_whole) / p.n_pieces;
+    const int merge_threads = n_split * kQBlock * (D / 8);
+    fa_merge_kernel<T, D><<<(merge_threads + kMergeThreads - 1) / kMergeThreads, kMergeThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -739,6 +949,25 @@ cudaError_t make_sm100_tmaps(const FaParams& p, TmaDesc* tq, TmaDesc* tk, TmaDes
     if (e == cudaSuccess) e = encode(tk, p, p.k, p.Tkv, p.Nkv, p.k_s, p.k_n, p.k_b);
     if (e == cudaSuccess) e = encode(tv, p, p.v, p.Tkv, p.Nkv, p.v_s, p.v_n, p.v_b);
     return e;
+}
+
+uint64_t plan_sm100_schedule(FaParams& p, int num_sms, bool uniform, int item_kv_blocks) {
+    p.grid = p.n_items < num_sms ? p.n_items : num_sms;
+    p.n_whole = p.n_tickets = p.n_items;
+    p.n_pieces = 0;
+    p.dynamic = uniform ? 0 : 1;  // unequal items: CTAs take the next ticket when free
+    if (!uniform || p.grid <= 0 || p.n_items <= p.grid) return 0;
+    // Equal items leave a last wave of n_items % grid items on a few SMs; split
+    // those items into key pieces so that the last wave spreads over the grid.
+    const int tail = p.n_items % p.grid;
+    if (tail == 0) return 0;
+    int pieces = p.grid / tail;
+    if (pieces > item_kv_blocks) pieces = item_kv_blocks;
+    if (pieces < 2) return 0;
+    p.n_whole = p.n_items - tail;
+    p.n_pieces = pieces;
+    p.n_tickets = p.n_whole + tail * pieces;
+    return static_cast<uint64_t>(tail) * pieces * kQBlock * (p.D + 4) * sizeof(float);
 }
 
 cudaError_t launch_sm100(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, const TmaDesc& tv, int num_sms,

@@ -18,10 +18,10 @@
 // array (kScratchBytes, about 130 KB) lives on every GPU that loads the
 // library until the process exits.
 //
-// The array is shared by every call: each call overwrites the offsets and
-// table it reads, so nothing has to start at zero, but two calls whose work
-// overlaps on the GPU (different streams, or different host threads without
-// ordering between them) race on it.
+// The array is shared by every call: each call overwrites the ticket counter
+// (with zero), the offsets and the table it reads, so nothing has to start at
+// zero, but two calls whose work overlaps on the GPU (different streams, or
+// different host threads without ordering between them) race on it.
 #include "fa_fwd.h"
 #include "fa_params.h"
 
@@ -34,8 +34,9 @@ namespace {
 
 constexpr int64_t kStaticMaxSeqs = 2048;
 constexpr int64_t kStaticMaxBlocks = (int64_t(1) << 20) / 256 + kStaticMaxSeqs;
+constexpr size_t kCuOffset = 256;  // [0, 256): the tcgen05 kernel's ticket counter
 constexpr size_t kCuBytes = 2 * (kStaticMaxSeqs + 1) * sizeof(int64_t);
-constexpr size_t kTableOffset = (kCuBytes + 255) & ~size_t(255);
+constexpr size_t kTableOffset = (kCuOffset + kCuBytes + 255) & ~size_t(255);
 constexpr size_t kScratchBytes = kTableOffset + kStaticMaxBlocks * sizeof(int4);
 constexpr int kMaxDevices = 64;
 
@@ -192,10 +193,11 @@ extern "C" fa_status fa_fwd_varlen_static(
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     unsigned char* dev = static_cast<unsigned char*>(scratch);
 
-    size_t bytes = kCuBytes;
+    size_t bytes = kCuOffset + kCuBytes;
     {
         std::lock_guard<std::mutex> lock(g_stage_mutex);
-        int64_t* cu = reinterpret_cast<int64_t*>(g_host_stage);
+        std::memset(g_host_stage, 0, kCuOffset);  // ticket counter = 0
+        int64_t* cu = reinterpret_cast<int64_t*>(g_host_stage + kCuOffset);
         cu[0] = 0;
         cu[nSeq + 1] = 0;
         for (int64_t b = 0; b < nSeq; ++b) {
@@ -225,7 +227,7 @@ extern "C" fa_status fa_fwd_varlen_static(
         if (cudaMemcpyAsync(dev, g_host_stage, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
             return FA_ERR_CUDA;
     }
-    p.cu_q = reinterpret_cast<const int64_t*>(dev);
+    p.cu_q = reinterpret_cast<const int64_t*>(dev + kCuOffset);
     p.cu_kv = p.cu_q + (nSeq + 1);
     cudaError_t err;
     if (sm100) {
@@ -234,9 +236,11 @@ extern "C" fa_status fa_fwd_varlen_static(
         if (cudaGetDevice(&device) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
             return FA_ERR_CUDA;
+        fa::plan_sm100_schedule(p, sms, false, 0);  // varlen items differ in cost: no split
+        p.sched_counter = reinterpret_cast<int*>(dev);
         fa::TmaDesc tq, tk, tv;
         if (fa::make_sm100_tmaps(p, &tq, &tk, &tv) != cudaSuccess) return FA_ERR_CUDA;
-        err = fa::launch_sm100(p, tq, tk, tv, sms, st);
+        err = fa::launch_sm100(p, tq, tk, tv, p.grid, st);
     } else {
         err = fa::launch_simt(p, st);
     }

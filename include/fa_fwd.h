@@ -19,8 +19,17 @@
  * Two-stage call, as on both operator pages ("接口原型" / "函数原型"):
  *   1. fa_fwd_get_workspace_size() validates every argument on the host, plans
  *      the launch and returns the device workspace size and an executor.  It
- *      makes no CUDA call and touches no device memory.
+ *      touches no device memory and enqueues nothing; its only CUDA calls read
+ *      the current device's SM count (cudaGetDevice, cudaDeviceGetAttribute),
+ *      and without a device it plans for a 148-SM B200.
  *   2. fa_fwd() enqueues the work on `stream` and consumes the executor.
+ *
+ * Workspace contents (tcgen05 kernel; the CUDA-core kernel needs none): a
+ * ticket counter (zeroed by fa_fwd on the stream when the schedule uses it),
+ * for TND the cumulative offsets and the list of work items, and, when the
+ * last wave of equal-cost work items is split along the keys, the pieces'
+ * partial results (fp32 O rows with their max and sum) that a second, small
+ * kernel merges.  Nothing in it has to be initialised by the caller.
  *
  * All floating-point accumulation is fp32.  Q·Kᵀ and P·V run on the tcgen05
  * tensor cores for fp16/bf16 inputs with head dim 64 or 128; fp32 inputs (and

@@ -80,7 +80,8 @@ def test_plan_half_types_use_tcgen05(layout, shape, n, dtype, d):
     q, k, v = qkv(shape, dtype)
     st, ws, text = fa.plan(q, k, v, input_layout=layout, head_num=n)
     assert st == 0, _abi.status_string(st)
-    assert "kernel=sm100_tcgen05" in text and f"D={d}" in text and ws == 0
+    # the workspace holds the ticket counter of the dynamic schedule
+    assert "kernel=sm100_tcgen05" in text and f"D={d}" in text and ws == 256
 
 
 def test_plan_varlen_workspace_holds_lengths_and_table():
@@ -93,7 +94,51 @@ def test_plan_varlen_workspace_holds_lengths_and_table():
     blocks = sum((x + 255) // 256 for x in lens)
     assert "kernel=sm100_tcgen05" in text and f"items={blocks * 24}" in text
     cu_bytes = (2 * (len(lens) + 1) * 8 + 255) // 256 * 256
-    assert ws == cu_bytes + blocks * 16
+    assert ws == 256 + cu_bytes + blocks * 16
+    assert "split_items=0" in text  # varlen items differ in cost: never split
+
+
+def _field(text, name):
+    return int(text.split(f"{name}=")[1].split()[0])
+
+
+def test_plan_splits_a_short_last_wave_of_equal_items():
+    # 149 equal items on 148 SMs: the last item is split into key pieces
+    # (at most one per 128-key block), each piece's partial rows kept in the
+    # workspace for the merge.
+    q, k, v = qkv((1, 149, 256, 128), torch.float16)
+    kk, vv = qkv((1, 149, 1024, 128), torch.float16)[1:]
+    st, ws, text = fa.plan(q, kk, vv, input_layout="BNSD", head_num=149)
+    assert st == 0, text
+    assert _field(text, "items") == 149 and _field(text, "grid") == 148
+    assert _field(text, "split_items") == 1 and _field(text, "pieces") == 8
+    assert ws == 256 + 1 * 8 * 256 * (128 + 4) * 4
+
+
+def test_plan_split_pieces_fill_the_grid():
+    # dense 2x24 heads x 16 query blocks = 768 items: 5 full waves + 28 items,
+    # split 148 // 28 = 5 ways
+    q, k, v = qkv((2, 24, 4096, 128), torch.float16)
+    st, ws, text = fa.plan(q, k, v, input_layout="BNSD", head_num=24)
+    assert st == 0
+    assert _field(text, "split_items") == 28 and _field(text, "pieces") == 5
+    assert ws == 256 + 28 * 5 * 256 * 132 * 4
+
+
+@pytest.mark.parametrize("kw", [dict(next_tokens=0), dict(pre_tokens=300, next_tokens=0)])
+def test_plan_does_not_split_unequal_items(kw):
+    # causal and banded items differ in cost (the band's first query blocks
+    # see fewer keys): the dynamic schedule balances them, nothing is split
+    q, k, v = qkv((1, 149, 1024, 128), torch.float16)
+    st, ws, text = fa.plan(q, k, v, input_layout="BNSD", head_num=149, **kw)
+    assert st == 0
+    assert _field(text, "split_items") == 0 and ws == 256
+
+
+def test_plan_no_split_when_items_fill_whole_waves():
+    q, k, v = qkv((1, 148, 512, 128), torch.float16)
+    st, ws, text = fa.plan(q, k, v, input_layout="BNSD", head_num=148)
+    assert st == 0 and _field(text, "items") == 296 and _field(text, "split_items") == 0
 
 
 def test_plan_unaligned_stride_falls_to_cuda_core_kernel():

@@ -12,7 +12,7 @@ from workloads import Workload, normal
 
 pytestmark = pytest.mark.gpu
 
-KNOWN_SITES = set(range(1, 10))
+KNOWN_SITES = set(range(1, 11))
 
 
 def small():

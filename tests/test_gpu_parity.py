@@ -273,3 +273,51 @@ def test_full_size_workloads_sampled(number):
     for t in res:
         assert not torch.isnan(t).any()
     compare_rows(w, res, sample_rows(w, 24, seed=number))
+
+
+# ---------------------------------------------------------------------------
+# Dynamic schedule: equal work items whose last wave is split into key pieces
+# and merged (the describe string says how many items were split)
+# ---------------------------------------------------------------------------
+
+def _split_of(w):
+    text = plan_text(w)
+    return int(text.split("split_items=")[1].split()[0]), int(text.split("pieces=")[1].split()[0])
+
+
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_split_last_wave_dense(dtype):
+    n = _sms() + 1  # one item past a full wave: that item is split into 8 key pieces
+    w = W("BNSD", dtype, (1, n, 256, 128), n, 3000, kshape=(1, n, 1024, 128))
+    assert _split_of(w) == (1, 8)
+    res = run_gpu(w)
+    compare_full(w, res)
+    again = run_gpu(w)
+    for a, b in zip(res, again):  # the merge order is fixed: bitwise reruns
+        assert torch.equal(a, b)
+
+
+def test_split_with_sink_gqa_and_ragged_keys():
+    n = _sms() + 2
+    nkv = n // 2 if n % 2 == 0 else n
+    w = W("BNSD", "bf16", (1, n, 256, 64), n, 3100, kshape=(1, nkv, 1000, 64), sink=normal((n,), "f32", 3104))
+    items, pieces = _split_of(w)
+    assert items == 2 and pieces == 8  # 1000 keys: 8 blocks, the last one ragged
+    compare_full(w)
+
+
+def test_split_random_mask_with_rows_empty_in_some_pieces():
+    n = _sms() + 1
+    sq, skv = 256, 1024
+    w = W("BNSD", "f16", (1, n, sq, 128), n, 3200, kshape=(1, n, skv, 128))
+    g = torch.Generator().manual_seed(3205)
+    mask = (torch.rand(1, 1, sq, skv, generator=g) < 0.4).to(torch.uint8)
+    mask[:, :, :10, : skv // 2] = 1   # rows 0-9: no key in the pieces over the first half
+    mask[:, :, 20, :] = 1             # row 20: no key at all (o = 0, m = -inf, l = 0)
+    w.atten_mask = mask
+    assert _split_of(w) == (1, 8)
+    compare_full(w)
