@@ -269,8 +269,8 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
         if (ticket == kTicketAbort) { ok = false; break; }
         if (ticket == kTicketEnd) break;
         const Work wk = work_of(p, ticket);
-        const Item& it = wk.it;
-        const TileRange* tr = wk.tr;
+        const Item it = wk.it;
+        const TileRange tr[2] = {wk.tr[0], wk.tr[1]};
         if (!tr[0].active() && !tr[1].active()) continue;
         const int lo = tr[0].active() ? (tr[1].active() ? min(tr[0].lo, tr[1].lo) : tr[0].lo) : tr[1].lo;
         const int hi = tr[0].active() ? (tr[1].active() ? max(tr[0].hi, tr[1].hi) : tr[0].hi) : tr[1].hi;
@@ -374,7 +374,7 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
         if (ticket == kTicketAbort) { ok = false; break; }
         if (ticket == kTicketEnd) break;
         const Work wk = work_of(p, ticket);
-        const TileRange* tr = wk.tr;
+        const TileRange tr[2] = {wk.tr[0], wk.tr[1]};
         if (!tr[0].active() && !tr[1].active()) continue;
         const int lo = tr[0].active() ? (tr[1].active() ? min(tr[0].lo, tr[1].lo) : tr[0].lo) : tr[1].lo;
         const int hi = tr[0].active() ? (tr[1].active() ? max(tr[0].hi, tr[1].hi) : tr[0].hi) : tr[1].hi;
@@ -543,8 +543,8 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, vo
         if (ticket == kTicketAbort) { ok = false; break; }
         if (ticket == kTicketEnd) break;
         const Work wk = work_of(p, ticket);
-        const Item& it = wk.it;
-        const TileRange tr = wk.tr[t];
+        const Item it = wk.it;
+        const TileRange tr = t ? wk.tr[1] : wk.tr[0];  // a select: no indexing of wk by a runtime value
         if (!tr.valid) continue;
         const int r0 = it.qb * kQBlock + t * kTileM;
         const int i = r0 + row;
