@@ -155,7 +155,7 @@ def plan(query, key, value, *, input_layout, head_num, scale=None, real_shift=No
          atten_mask=None, mask_mode=FA_MASK_TENSOR, sink=None, actual_seq_qlen=None,
          actual_seq_kvlen=None, pre_tokens=INT64_MAX, next_tokens=INT64_MAX, keep_prob=1.0,
          inner_precise=0, softmax_out_layout="", out=None, softmax_max=None, softmax_sum=None):
-    """Stage 1 only (no CUDA call): returns (status, workspace_bytes, plan_text)."""
+    """Stage 1 only (no device work): returns (status, workspace_bytes, plan_text)."""
     _, dv, scale, pse_type = _defaults(query, key, value, input_layout, head_num, scale, real_shift, pse_type)
     out_shape, stats_shape = _out_shapes(query, input_layout, head_num, dv, softmax_out_layout)
     dev = query.device
