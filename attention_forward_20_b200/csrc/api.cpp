@@ -321,6 +321,9 @@ extern "C" fa_status fa_fwd_get_workspace_size(
     p.mask_cols = attenMask ? (int32_t)attenMask->shape[attenMask->ndim - 1] : 0;
     auto aligned16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; };
     p.o_vec = aligned16(p.o) && p.o_b % 8 == 0 && p.o_n % 8 == 0 && p.o_s % 8 == 0;
+    auto aligned32 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 31u) == 0; };
+    p.o_vec32 = aligned32(p.o) && p.o_b % 16 == 0 && p.o_n % 16 == 0 && p.o_s % 16 == 0;
+    p.st_vec32 = aligned32(p.smax) && aligned32(p.ssum) && p.st_b % 8 == 0 && p.st_n % 8 == 0 && p.st_s % 8 == 0;
     p.mask_vec = attenMask && aligned16(p.mask) && p.mask_b % 16 == 0 && p.mask_n % 16 == 0 && p.mask_i % 16 == 0;
     p.pse_vec = realShift && pseType == FA_PSE_DENSE && aligned16(p.pse) && p.pse_b % 8 == 0 &&
                 p.pse_n % 8 == 0 && p.pse_i % 8 == 0;

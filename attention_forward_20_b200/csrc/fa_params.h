@@ -54,6 +54,8 @@ struct FaParams {
     int32_t Tq, Tkv;            // rows of the query / key tensors (TND: packed tokens; else Sq / Skv)
     int32_t mask_cols;          // allocated width of a mask row (columns readable from mask)
     int32_t o_vec;              // output rows allow 16-byte stores
+    int32_t o_vec32;            // output rows allow 32-byte stores
+    int32_t st_vec32;           // the 8 lanes of a statistics row allow 32-byte stores
     int32_t mask_vec;           // mask rows allow 16-byte loads
     int32_t pse_vec;            // dense bias rows allow 16-byte loads
     int32_t debug_stall;        // failure injection: the MMA warp waits on a barrier never signalled

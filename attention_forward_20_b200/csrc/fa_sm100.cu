@@ -99,6 +99,12 @@ struct Item {
     int64_t q_off, kv_off;
 };
 
+// The dynamic schedule's hand-off slots: the ticket and its decoded item (the
+// TMA warp pays for the varlen table and offset loads, the others read smem).
+struct TicketSlots {
+    Item item[kSched];
+};
+
 // Work item -> (batch, head, query block).  Dense layouts: groups of
 // kHeadGroup heads; inside a group the query blocks go from the last (the
 // most keys under a causal band) to the first, heads fastest.  TND: the host
@@ -168,18 +174,20 @@ struct Work {
     int tail;
 };
 
-__device__ __forceinline__ Work work_of(const FaParams& p, int ticket) {
+__device__ __forceinline__ int item_of_ticket(const FaParams& p, int ticket) {
+    return ticket < p.n_whole ? ticket : p.n_whole + (ticket - p.n_whole) / p.n_pieces;
+}
+
+__device__ __forceinline__ Work work_of(const FaParams& p, int ticket, const Item& it) {
     Work w;
-    int item = ticket;
     w.piece = -1;
     w.tail = 0;
     if (ticket >= p.n_whole) {
         const int u = ticket - p.n_whole;
         w.tail = u / p.n_pieces;
         w.piece = u - w.tail * p.n_pieces;
-        item = p.n_whole + w.tail;
     }
-    w.it = decode_item(p, item);
+    w.it = it;
     w.tr[0] = tile_range(p, w.it, 0);
     w.tr[1] = tile_range(p, w.it, 1);
     if (w.piece >= 0 && (w.tr[0].active() || w.tr[1].active())) {
@@ -212,29 +220,39 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 // Otherwise the TMA warp takes the next ticket from the global counter as soon
 // as it has issued the loads of the previous one, and hands it to the MMA warp
 // and the softmax warps through kSched shared-memory slots.
-__device__ __forceinline__ int static_ticket(const FaParams& p, uint32_t& k) {
+__device__ __forceinline__ int static_ticket(const FaParams& p, uint32_t& k, Item& it) {
     const int tk = blockIdx.x + static_cast<int>(k++) * gridDim.x;
-    return tk < p.n_tickets ? tk : kTicketEnd;
+    if (tk >= p.n_tickets) return kTicketEnd;
+    it = decode_item(p, item_of_ticket(p, tk));
+    return tk;
 }
-__device__ __forceinline__ int take_ticket_global(const FaParams& p, Barriers& bars, uint32_t& k, volatile int* abort) {
-    if (!p.dynamic) return static_ticket(p, k);
+__device__ __forceinline__ int take_ticket_global(const FaParams& p, Barriers& bars, TicketSlots& slots, uint32_t& k,
+                                                  Item& it, volatile int* abort) {
+    if (!p.dynamic) return static_ticket(p, k, it);
     const uint32_t slot = k % kSched;
     if (!warp_wait(&bars.sched_empty[slot], ((k / kSched) & 1) ^ 1, abort, kSiteSched)) return kTicketAbort;
     int tk = 0;
     if ((threadIdx.x & 31) == 0) {
         tk = atomicAdd(p.sched_counter, 1);
         if (tk >= p.n_tickets) tk = kTicketEnd;
+    }
+    tk = __shfl_sync(0xffffffffu, tk, 0);
+    if (tk >= 0) it = decode_item(p, item_of_ticket(p, tk));
+    if ((threadIdx.x & 31) == 0) {
         bars.ticket[slot] = tk;
+        if (tk >= 0) slots.item[slot] = it;
         mbar_arrive(&bars.sched_full[slot]);
     }
     ++k;
-    return __shfl_sync(0xffffffffu, tk, 0);
+    return tk;
 }
-__device__ __forceinline__ int take_ticket_local(const FaParams& p, Barriers& bars, uint32_t& k, volatile int* abort) {
-    if (!p.dynamic) return static_ticket(p, k);
+__device__ __forceinline__ int take_ticket_local(const FaParams& p, Barriers& bars, const TicketSlots& slots,
+                                                 uint32_t& k, Item& it, volatile int* abort) {
+    if (!p.dynamic) return static_ticket(p, k, it);
     const uint32_t slot = k % kSched;
     if (!warp_wait(&bars.sched_full[slot], (k / kSched) & 1, abort, kSiteSched)) return kTicketAbort;
     const int tk = *reinterpret_cast<volatile int*>(&bars.ticket[slot]);
+    if (tk >= 0) it = slots.item[slot];
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(&bars.sched_empty[slot]);
     ++k;
@@ -248,7 +266,7 @@ __device__ __forceinline__ int take_ticket_local(const FaParams& p, Barriers& ba
 template <int D>
 __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
                              const CUtensorMap* tv, uint8_t* sQ, uint8_t* sKV, Barriers& bars,
-                             volatile int* abort) {
+                             TicketSlots& slots, volatile int* abort) {
     using C = Cfg<D>;
     uint32_t kv_fill = 0, q_fill[2] = {0, 0}, k_sched = 0;
     bool ok = true;
@@ -265,10 +283,11 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
     };
 
     while (ok) {
-        const int ticket = take_ticket_global(p, bars, k_sched, abort);
+        Item tit;
+        const int ticket = take_ticket_global(p, bars, slots, k_sched, tit, abort);
         if (ticket == kTicketAbort) { ok = false; break; }
         if (ticket == kTicketEnd) break;
-        const Work wk = work_of(p, ticket);
+        const Work wk = work_of(p, ticket, tit);
         const Item it = wk.it;
         const TileRange tr[2] = {wk.tr[0], wk.tr[1]};
         if (!tr[0].active() && !tr[1].active()) continue;
@@ -327,8 +346,8 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
 // same lane every time, so its commits cover its MMAs)
 // ---------------------------------------------------------------------------
 template <typename T, int D>
-__device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& bars, uint32_t tmem,
-                        volatile int* abort) {
+__device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& bars, const TicketSlots& slots,
+                        uint32_t tmem, volatile int* abort) {
     using C = Cfg<D>;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     const uint32_t idesc_qk = idesc_f16(kBf16, kTileM, kTileN, false, false, p.neg_scale != 0);
@@ -370,10 +389,11 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
     };
 
     while (ok) {
-        const int ticket = take_ticket_local(p, bars, k_sched, abort);
+        Item tit;
+        const int ticket = take_ticket_local(p, bars, slots, k_sched, tit, abort);
         if (ticket == kTicketAbort) { ok = false; break; }
         if (ticket == kTicketEnd) break;
-        const Work wk = work_of(p, ticket);
+        const Work wk = work_of(p, ticket, tit);
         const TileRange tr[2] = {wk.tr[0], wk.tr[1]};
         if (!tr[0].active() && !tr[1].active()) continue;
         const int lo = tr[0].active() ? (tr[1].active() ? min(tr[0].lo, tr[1].lo) : tr[0].lo) : tr[1].lo;
@@ -498,7 +518,10 @@ __device__ __forceinline__ void store_out32(const FaParams& p, T* orow, int cc, 
 #pragma unroll
     for (int e = 0; e < 16; ++e)
         w[e] = pack2<T>(__uint_as_float(o[2 * e]) * o_scale, __uint_as_float(o[2 * e + 1]) * o_scale);
-    if (p.o_vec) {
+    if (p.o_vec32) {  // whole 32-byte sectors: half the store requests of 16-byte stores
+        st_global_v8(orow + cc, w);
+        st_global_v8(orow + cc + 16, w + 8);
+    } else if (p.o_vec) {
         uint4* dst = reinterpret_cast<uint4*>(orow + cc);
 #pragma unroll
         for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
@@ -519,6 +542,17 @@ __device__ __forceinline__ void store_out32(const FaParams& p, T* orow, int cc, 
 __device__ __forceinline__ void store_stats(const FaParams& p, const Item& it, int i, const RowFinal& f) {
     const int64_t so = it.b * p.st_b + it.n * p.st_n + (it.q_off + i) * p.st_s;
     const float m_nat = f.m_f * kLn2;
+    if (p.st_vec32) {
+        uint32_t wm[8], wl[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            wm[e] = __float_as_uint(m_nat);
+            wl[e] = __float_as_uint(f.l_f);
+        }
+        st_global_v8(p.smax + so, wm);
+        st_global_v8(p.ssum + so, wl);
+        return;
+    }
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
         p.smax[so + e] = m_nat;
@@ -526,8 +560,11 @@ __device__ __forceinline__ void store_stats(const FaParams& p, const Item& it, i
     }
 }
 
-template <typename T, int D, bool kBias>
-__device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, volatile int* abort, int t) {
+// kBias: 0 no bias, 1 dense bias tensor, 2 ALiBi slopes (one variant each, so
+// that each kernel carries only its own bias code).
+template <typename T, int D, int kBias>
+__device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots& slots, uint32_t tmem,
+                            volatile int* abort, int t) {
     using C = Cfg<D>;
     const int quad = (threadIdx.x >> 5) & 3;
     const int row = quad * 32 + (threadIdx.x & 31);
@@ -539,10 +576,11 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, vo
     bool ok = true;
 
     while (ok) {
-        const int ticket = take_ticket_local(p, bars, k_sched, abort);
+        Item tit;
+        const int ticket = take_ticket_local(p, bars, slots, k_sched, tit, abort);
         if (ticket == kTicketAbort) { ok = false; break; }
         if (ticket == kTicketEnd) break;
-        const Work wk = work_of(p, ticket);
+        const Work wk = work_of(p, ticket, tit);
         const Item it = wk.it;
         const TileRange tr = t ? wk.tr[1] : wk.tr[0];  // a select: no indexing of wk by a runtime value
         if (!tr.valid) continue;
@@ -552,12 +590,11 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, vo
 
         float slope_l2 = 0.f;
         const T* pse_row = nullptr;
-        if (kBias) {
-            if (p.pse_type == 2)
-                slope_l2 = static_cast<const float*>(p.pse)[it.b * p.pse_b + it.n * p.pse_n] * kLog2e;
-            else if (row_ok)
+        if constexpr (kBias == 2)
+            slope_l2 = static_cast<const float*>(p.pse)[it.b * p.pse_b + it.n * p.pse_n] * kLog2e;
+        if constexpr (kBias == 1)
+            if (row_ok)
                 pse_row = static_cast<const T*>(p.pse) + it.b * p.pse_b + it.n * p.pse_n + (int64_t)i * p.pse_i;
-        }
         const uint8_t* mask_row =
             (p.mask_on && row_ok) ? p.mask + it.b * p.mask_b + it.n * p.mask_n + (int64_t)i * p.mask_i : nullptr;
 
@@ -584,7 +621,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, vo
 #pragma unroll
                 for (int c8 = 0; c8 < kTileN; c8 += 8) {
                     float bias[8];
-                    if (p.pse_type == 2) {
+                    if constexpr (kBias == 2) {
 #pragma unroll
                         for (int e = 0; e < 8; ++e) bias[e] = -slope_l2 * fabsf(fi - (float)(c8 + e));
                     } else if (pse_row) {
@@ -677,7 +714,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, vo
             // row's m_run, m_used, l for the merge.
             float* prow = p.part + ((static_cast<size_t>(wk.tail) * p.n_pieces + wk.piece) * kQBlock + t * kTileM + row) *
                                        static_cast<size_t>(D + 4);
-#pragma unroll
+#pragma unroll 1
             for (int cc = 0; cc < D; cc += 32) {
                 uint32_t o[32];
                 if (has_blocks) {
@@ -697,7 +734,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, uint32_t tmem, vo
         }
         const RowFinal f = finalize_row(p, it, m_run, m_used, l);
         T* orow = static_cast<T*>(p.o) + it.b * p.o_b + it.n * p.o_n + (it.q_off + i) * p.o_s;
-#pragma unroll
+#pragma unroll 1
         for (int cc = 0; cc < D; cc += 32) {
             uint32_t o[32];
             if (has_blocks) {
@@ -779,7 +816,7 @@ __global__ void __launch_bounds__(kMergeThreads) fa_merge_kernel(const FaParams 
 // ---------------------------------------------------------------------------
 // Kernel
 // ---------------------------------------------------------------------------
-template <typename T, int D, bool kBias>
+template <typename T, int D, int kBias>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, const FaParams p) {
@@ -789,6 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sQ = smem;
     uint8_t* sKV = smem + 2 * C::kTileBytes;
     __shared__ Barriers bars;
+    __shared__ TicketSlots slots;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
 
@@ -830,13 +868,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 8) {
         setmaxnreg_inc<kSoftmaxRegs>();
-        run_softmax<T, D, kBias>(p, bars, tmem, &abort_flag, warp >> 2);
+        run_softmax<T, D, kBias>(p, bars, slots, tmem, &abort_flag, warp >> 2);
     } else {
         setmaxnreg_dec<kOtherRegs>();
         if (warp == kLoadWarp)
-            run_producer<D>(p, &tmap_q, &tmap_k, &tmap_v, sQ, sKV, bars, &abort_flag);
+            run_producer<D>(p, &tmap_q, &tmap_k, &tmap_v, sQ, sKV, bars, slots, &abort_flag);
         else if (warp == kMmaWarp)
-            run_mma<T, D>(p, sQ, sKV, bars, tmem, &abort_flag);
+            run_mma<T, D>(p, sQ, sKV, bars, slots, tmem, &abort_flag);
     }
 
     tc_fence_before();
@@ -847,7 +885,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicCAS(&g_fa_error, 0ull, (static_cast<unsigned long long>(abort_flag) << 32) | (blockIdx.x + 1u));
 }
 
-template <typename T, int D, bool kBias>
+template <typename T, int D, int kBias>
 cudaError_t launch_t(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, const TmaDesc& tv, int num_sms,
                      cudaStream_t stream) {
     using C = Cfg<D>;
@@ -878,12 +916,15 @@ cudaError_t launch_t(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, co
 template <typename T>
 cudaError_t launch_d(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, const TmaDesc& tv, int num_sms,
                      cudaStream_t stream) {
-    const bool bias = p.pse_type != 0;
-    if (p.D == 128)
-        return bias ? launch_t<T, 128, true>(p, tq, tk, tv, num_sms, stream)
-                    : launch_t<T, 128, false>(p, tq, tk, tv, num_sms, stream);
-    return bias ? launch_t<T, 64, true>(p, tq, tk, tv, num_sms, stream)
-                : launch_t<T, 64, false>(p, tq, tk, tv, num_sms, stream);
+    // pse_type is 0 whenever realShift is absent
+    if (p.D == 128) {
+        if (p.pse_type == 2) return launch_t<T, 128, 2>(p, tq, tk, tv, num_sms, stream);
+        if (p.pse_type == 1) return launch_t<T, 128, 1>(p, tq, tk, tv, num_sms, stream);
+        return launch_t<T, 128, 0>(p, tq, tk, tv, num_sms, stream);
+    }
+    if (p.pse_type == 2) return launch_t<T, 64, 2>(p, tq, tk, tv, num_sms, stream);
+    if (p.pse_type == 1) return launch_t<T, 64, 1>(p, tq, tk, tv, num_sms, stream);
+    return launch_t<T, 64, 0>(p, tq, tk, tv, num_sms, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -172,6 +172,9 @@ extern "C" fa_status fa_fwd_varlen_static(
     p.Tq = (int32_t)Tq; p.Tkv = (int32_t)Tk;
     auto aligned16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; };
     p.o_vec = aligned16(p.o) && p.o_n % 8 == 0 && p.o_s % 8 == 0;
+    auto aligned32 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 31u) == 0; };
+    p.o_vec32 = aligned32(p.o) && p.o_n % 16 == 0 && p.o_s % 16 == 0;
+    p.st_vec32 = aligned32(p.smax) && aligned32(p.ssum) && p.st_n % 8 == 0 && p.st_s % 8 == 0;
     auto tma_dim_ok = [](int64_t stride, int64_t size) {
         return size == 1 || (stride > 0 && (stride * 2) % 16 == 0 && stride * 2 < (int64_t(1) << 40));
     };
