@@ -635,16 +635,24 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                 }
             }
             if (!full) {
+                // keys of this row kept by the sequence end and the band:
+                // columns [c_lo, c_hi] of the block (empty when c_hi < c_lo)
+                const int c_lo = max(0, i - p.pre - j0);
+                const int c_hi = min(min(kTileN - 1, it.kv_len - 1 - j0), i + p.next - j0);
+                if (mask_row) {
 #pragma unroll
-                for (int c16 = 0; c16 < kTileN; c16 += 16) {
-                    const uint32_t excl = mask_row ? load_mask16(mask_row, j0 + c16, p.mask_cols, p.mask_vec != 0) : 0u;
+                    for (int c16 = 0; c16 < kTileN; c16 += 16) {
+                        const uint32_t excl = load_mask16(mask_row, j0 + c16, p.mask_cols, p.mask_vec != 0);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int j = j0 + c16 + e;
-                        const int d = j - i;
-                        const bool keep = j < it.kv_len && d >= -p.pre && d <= p.next && !((excl >> e) & 1u);
-                        if (!keep) s[c16 + e] = -CUDART_INF_F;
+                        for (int e = 0; e < 16; ++e) {
+                            const int c = c16 + e;
+                            if (c < c_lo || c > c_hi || ((excl >> e) & 1u)) s[c] = -CUDART_INF_F;
+                        }
                     }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < kTileN; ++c)
+                        if (c < c_lo || c > c_hi) s[c] = -CUDART_INF_F;
                 }
             }
             {
