@@ -9,10 +9,13 @@
 // produces are those of the forward and sink formulas on the
 // aclnnFlashAttentionVarLenScoreV5 page.
 //
-// CTA = 128 threads = 4 warps for 32 query rows (8 rows per warp).  For each
-// 32-key tile staged in shared memory, lane j of a warp scores key j against
-// one row, the warp reduces the row max and sum with shuffles, and every lane
-// accumulates its D/32 output columns.
+// CTA = 8 warps, one query row per warp.  Keys go in tiles of kKeys (128, or
+// 64 when the head dim exceeds 128) staged in shared memory as fp32; lane l
+// scores keys l, l+32, ... (independent FMA chains over the head dim), the
+// warp reduces the row max once per tile, keeps its share of the row sum in
+// each lane (reduced once at the end), writes P to shared memory and
+// accumulates its output columns d = l + 32t over the tile's keys with four
+// interleaved partial sums.
 #include "fa_params.h"
 
 #include <cuda_bf16.h>
@@ -22,10 +25,8 @@
 namespace fa {
 namespace {
 
-constexpr int kRows = 32;  // query rows per CTA
-constexpr int kKeys = 32;  // keys per tile (one per lane)
-constexpr int kWarps = 4;
-constexpr int kRowsPerWarp = kRows / kWarps;
+constexpr int kWarps = 8;
+constexpr int kRows = kWarps;  // query rows per CTA, one per warp
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
@@ -47,14 +48,24 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+template <int DMAX>
+struct SimtCfg {
+    static constexpr int kKeys = DMAX <= 128 ? 128 : 64;  // keys per tile
+    static constexpr int kPerLane = kKeys / 32;
+    static constexpr int kCols = DMAX / 32;               // output columns per lane
+    static constexpr int ld = DMAX + 1;                   // odd pitch: lane-strided rows hit distinct banks
+    static constexpr size_t kSmemBytes = size_t(2 * kKeys * ld + kRows * ld + kRows * kKeys) * sizeof(float);
+};
+
 template <typename T, int DMAX>
-__global__ void __launch_bounds__(kWarps * 32) fa_fwd_simt_kernel(const FaParams p) {
+__global__ void __launch_bounds__(kWarps * 32, 1) fa_fwd_simt_kernel(const FaParams p) {
+    using C = SimtCfg<DMAX>;
+    constexpr int kKeys = C::kKeys, kPerLane = C::kPerLane, kCols = C::kCols, ld = C::ld;
     extern __shared__ float smem[];
-    constexpr int ld = DMAX + 1;  // odd row pitch: lane-strided reads hit distinct banks
-    constexpr int kCols = DMAX / 32;
-    float* sQ = smem;
-    float* sK = sQ + kRows * ld;
-    float* sV = sK + kKeys * ld;
+    float* sK = smem;                  // [kKeys][ld]
+    float* sV = sK + kKeys * ld;       // [kKeys][ld]
+    float* sQ = sV + kKeys * ld;       // [kRows][ld]
+    float* sP = sQ + kRows * ld;       // [kRows][kKeys]
 
     const int b = blockIdx.z, n = blockIdx.y, i0 = blockIdx.x * kRows;
     const int nk = n / p.group;
@@ -73,19 +84,13 @@ __global__ void __launch_bounds__(kWarps * 32) fa_fwd_simt_kernel(const FaParams
     const T* V = static_cast<const T*>(p.v) + b * p.v_b + nk * p.v_n;
     const int D = p.D, Dv = p.Dv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int i = i0 + warp;  // this warp's query row
+    const bool row_ok = i < q_len;
 
-    for (int idx = tid; idx < kRows * D; idx += blockDim.x) {
-        const int r = idx / D, d = idx % D, i = i0 + r;
-        sQ[r * ld + d] = (i < q_len) ? to_f(Q[(q_off + i) * p.q_s + d]) : 0.f;
-    }
-
-    float m[kRowsPerWarp], l[kRowsPerWarp], acc[kRowsPerWarp][kCols];
-#pragma unroll
-    for (int rr = 0; rr < kRowsPerWarp; ++rr) {
-        m[rr] = -CUDART_INF_F;
-        l[rr] = 0.f;
-#pragma unroll
-        for (int t = 0; t < kCols; ++t) acc[rr][t] = 0.f;
+    // Q rows, zero-padded to DMAX (the dot products run over DMAX)
+    for (int idx = tid; idx < kRows * DMAX; idx += blockDim.x) {
+        const int r = idx / DMAX, d = idx % DMAX, ii = i0 + r;
+        sQ[r * ld + d] = (ii < q_len && d < D) ? to_f(Q[(q_off + ii) * p.q_s + d]) : 0.f;
     }
 
     float slope = 0.f;
@@ -93,84 +98,128 @@ __global__ void __launch_bounds__(kWarps * 32) fa_fwd_simt_kernel(const FaParams
     const T* pse = (p.pse_type == 1) ? static_cast<const T*>(p.pse) + b * p.pse_b + n * p.pse_n : nullptr;
     const uint8_t* mask = p.mask_on ? p.mask + b * p.mask_b + n * p.mask_n : nullptr;
 
+    float m_run = -CUDART_INF_F, l_lane = 0.f;
+    float acc[4][kCols];
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+#pragma unroll
+        for (int t = 0; t < kCols; ++t) acc[g][t] = 0.f;
+
+    // keys any row of the CTA keeps under the band
     const int i1 = min(q_len, i0 + kRows) - 1;
     const int j_lo = max(0, i0 - p.pre);
     const int j_hi = min(kv_len - 1, i1 + p.next);
+    const float* q = sQ + warp * ld;
+    float* pw = sP + warp * kKeys;
     for (int j0 = (j_lo / kKeys) * kKeys; j0 <= j_hi; j0 += kKeys) {
         __syncthreads();
-        for (int idx = tid; idx < kKeys * D; idx += blockDim.x) {
-            const int r = idx / D, d = idx % D, j = j0 + r;
-            sK[r * ld + d] = (j < kv_len) ? to_f(K[(kv_off + j) * p.k_s + d]) : 0.f;
-        }
-        for (int idx = tid; idx < kKeys * Dv; idx += blockDim.x) {
-            const int r = idx / Dv, d = idx % Dv, j = j0 + r;
-            sV[r * ld + d] = (j < kv_len) ? to_f(V[(kv_off + j) * p.v_s + d]) : 0.f;
+        // K/V tile: batches of kBatch elements per thread, all loads of a batch
+        // in flight before their shared-memory stores
+        constexpr int kPerThread = kKeys * DMAX / (kWarps * 32);
+        constexpr int kBatch = 16;
+#pragma unroll 1
+        for (int u = 0; u < kPerThread; u += kBatch) {
+            float kk[kBatch], vv[kBatch];
+#pragma unroll
+            for (int e = 0; e < kBatch; ++e) {
+                const int idx = tid + (u + e) * (kWarps * 32);
+                const int r = idx / DMAX, d = idx % DMAX, j = j0 + r;
+                const bool in = j < kv_len;
+                kk[e] = (in && d < D) ? to_f(K[(kv_off + j) * p.k_s + d]) : 0.f;
+                vv[e] = (in && d < Dv) ? to_f(V[(kv_off + j) * p.v_s + d]) : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < kBatch; ++e) {
+                const int idx = tid + (u + e) * (kWarps * 32);
+                const int r = idx / DMAX, d = idx % DMAX;
+                sK[r * ld + d] = kk[e];
+                sV[r * ld + d] = vv[e];
+            }
         }
         __syncthreads();
-        const int j = j0 + lane;
+
+        // scores of keys j0 + lane + 32m
+        float x[kPerLane];
 #pragma unroll
-        for (int rr = 0; rr < kRowsPerWarp; ++rr) {
-            const int r = warp * kRowsPerWarp + rr, i = i0 + r;
-            float s = 0.f;
-            for (int d = 0; d < D; ++d) s = fmaf(sQ[r * ld + d], sK[lane * ld + d], s);
-            bool keep = i < q_len && j < kv_len && (j - i >= -p.pre) && (j - i <= p.next);
-            if (keep && mask) keep = mask[(int64_t)i * p.mask_i + j] == 0;
-            float x = s * p.scale;
-            if (keep && pse) x += to_f(pse[(int64_t)i * p.pse_i + j]);
-            if (p.pse_type == 2) x -= slope * fabsf((float)(i - j));
-            x = keep ? x : -CUDART_INF_F;
-            const float m_new = fmaxf(m[rr], warp_max(x));
-            if (m_new == -CUDART_INF_F) continue;  // nothing kept yet in this row
-            const float alpha = expf(m[rr] - m_new);
-            const float pj = keep ? expf(x - m_new) : 0.f;
-            l[rr] = l[rr] * alpha + warp_sum(pj);
+        for (int mm = 0; mm < kPerLane; ++mm) x[mm] = 0.f;
+#pragma unroll 8
+        for (int d = 0; d < DMAX; ++d) {
+            const float qd = q[d];
 #pragma unroll
-            for (int t = 0; t < kCols; ++t) acc[rr][t] *= alpha;
-            for (int jj = 0; jj < kKeys; ++jj) {
-                const float pv = __shfl_sync(0xffffffffu, pj, jj);
-#pragma unroll
-                for (int t = 0; t < kCols; ++t) {
-                    const int d = lane + 32 * t;
-                    if (d < Dv) acc[rr][t] = fmaf(pv, sV[jj * ld + d], acc[rr][t]);
-                }
-            }
-            m[rr] = m_new;
+            for (int mm = 0; mm < kPerLane; ++mm) x[mm] = fmaf(qd, sK[(lane + 32 * mm) * ld + d], x[mm]);
         }
+        float tile_max = -CUDART_INF_F;
+#pragma unroll
+        for (int mm = 0; mm < kPerLane; ++mm) {
+            const int j = j0 + lane + 32 * mm;
+            bool keep = row_ok && j < kv_len && (j - i >= -p.pre) && (j - i <= p.next);
+            if (keep && mask) keep = mask[(int64_t)i * p.mask_i + j] == 0;
+            float v = x[mm] * p.scale;
+            if (keep && pse) v += to_f(pse[(int64_t)i * p.pse_i + j]);
+            if (p.pse_type == 2) v -= slope * fabsf((float)(i - j));
+            x[mm] = keep ? v : -CUDART_INF_F;
+            tile_max = fmaxf(tile_max, x[mm]);
+        }
+        const float m_new = fmaxf(m_run, warp_max(tile_max));
+        if (m_new == -CUDART_INF_F) continue;  // nothing kept in this row yet (warp-uniform)
+        const float alpha = expf(m_run - m_new);  // 0 when m_run is -inf
+        m_run = m_new;
+        float psum = 0.f;
+#pragma unroll
+        for (int mm = 0; mm < kPerLane; ++mm) {
+            const float pj = expf(x[mm] - m_new);  // 0 for excluded keys
+            psum += pj;
+            pw[lane + 32 * mm] = pj;
+        }
+        l_lane = l_lane * alpha + psum;
+        __syncwarp();
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+#pragma unroll
+            for (int t = 0; t < kCols; ++t) acc[g][t] *= alpha;
+        // O += P V over the tile: four interleaved partial sums per column
+#pragma unroll 2
+        for (int jj = 0; jj < kKeys; jj += 4) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const float pj = pw[jj + g];
+#pragma unroll
+                for (int t = 0; t < kCols; ++t)
+                    acc[g][t] = fmaf(pj, sV[(jj + g) * ld + lane + 32 * t], acc[g][t]);
+            }
+        }
+        __syncwarp();
     }
 
-    T* O = static_cast<T*>(p.o) + b * p.o_b + n * p.o_n;
+    if (!row_ok) return;
+    const float l = warp_sum(l_lane);
+    float mf = m_run, lf = l, oscale;
+    if (p.has_sink) {
+        // sink formula: m = max(sink, max S); denominator gains e^(sink - m)
+        const float sk = p.sink[n];
+        mf = fmaxf(m_run, sk);
+        const float a = (m_run == -CUDART_INF_F) ? 0.f : expf(m_run - mf);
+        lf = l * a + expf(sk - mf);
+        oscale = a / lf;
+    } else {
+        oscale = lf > 0.f ? 1.f / lf : 0.f;
+    }
+    T* orow = static_cast<T*>(p.o) + b * p.o_b + n * p.o_n + (q_off + i) * p.o_s;
 #pragma unroll
-    for (int rr = 0; rr < kRowsPerWarp; ++rr) {
-        const int i = i0 + warp * kRowsPerWarp + rr;
-        if (i >= q_len) continue;
-        float mf = m[rr], lf = l[rr], oscale;
-        if (p.has_sink) {
-            // sink formula: m = max(sink, max S); denominator gains e^(sink - m)
-            const float sk = p.sink[n];
-            mf = fmaxf(m[rr], sk);
-            const float a = (m[rr] == -CUDART_INF_F) ? 0.f : expf(m[rr] - mf);
-            lf = l[rr] * a + expf(sk - mf);
-            oscale = a / lf;
-        } else {
-            oscale = lf > 0.f ? 1.f / lf : 0.f;
-        }
-        T* orow = O + (q_off + i) * p.o_s;
-#pragma unroll
-        for (int t = 0; t < kCols; ++t) {
-            const int d = lane + 32 * t;
-            if (d < Dv) orow[d] = from_f<T>(acc[rr][t] * oscale);
-        }
-        const int64_t so = b * p.st_b + n * p.st_n + (q_off + i) * p.st_s;
-        if (lane < 8) {
-            p.smax[so + lane] = mf;
-            p.ssum[so + lane] = lf;
-        }
+    for (int t = 0; t < kCols; ++t) {
+        const int d = lane + 32 * t;
+        if (d < Dv) orow[d] = from_f<T>(((acc[0][t] + acc[1][t]) + (acc[2][t] + acc[3][t])) * oscale);
+    }
+    const int64_t so = b * p.st_b + n * p.st_n + (q_off + i) * p.st_s;
+    if (lane < 8) {
+        p.smax[so + lane] = mf;
+        p.ssum[so + lane] = lf;
     }
 }
 
 template <typename T, int DMAX>
 cudaError_t launch_t(const FaParams& p, cudaStream_t stream) {
-    const size_t smem = size_t(kRows + 2 * kKeys) * (DMAX + 1) * sizeof(float);
+    const size_t smem = SimtCfg<DMAX>::kSmemBytes;
     auto kern = fa_fwd_simt_kernel<T, DMAX>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
