@@ -616,7 +616,33 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
 
             // scores in the log2 domain (bias path) and the block's row max
             float m_blk;
-            if constexpr (kBias) {
+            float row_off = 0.f;  // a per-row bias term kept out of s (added to the max and the shift)
+            bool linear = false;
+            if constexpr (kBias == 2) {
+                // A block wholly on one side of every row's diagonal has
+                // -slope·|i - j| = st·c - st·(i - j0) with st = ±slope: a ramp
+                // over the columns plus a per-row constant.
+                const bool below = j0 + kTileN - 1 <= r0;
+                const bool above = j0 >= r0 + kTileM - 1;
+                linear = below || above;
+                if (linear) {
+                    const float st = below ? slope_l2 : -slope_l2;
+                    row_off = -st * (float)(i - j0);
+                    float t[8];  // ramp at columns c8 + h, four chains of column pairs
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) t[h] = st * (float)h;
+                    const float step = 8.f * st;
+#pragma unroll
+                    for (int c8 = 0; c8 < kTileN; c8 += 8) {
+#pragma unroll
+                        for (int h = 0; h < 8; h += 2) {
+                            fma2(s[c8 + h], s[c8 + h + 1], s[c8 + h], s[c8 + h + 1], sl2, sl2, t[h], t[h + 1]);
+                            add2(t[h], t[h + 1], step, step);
+                        }
+                    }
+                }
+            }
+            if (kBias && !linear) {
                 const float fi = (float)(i - j0);
 #pragma unroll
                 for (int c8 = 0; c8 < kTileN; c8 += 8) {
@@ -656,12 +682,17 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                 }
             }
             {
-                // columns 0..3 seed four chains; pairs 4..127 feed them in turn
-                float mc[4] = {s[0], s[1], s[2], s[3]};
+                // eight chains: columns 0..15 seed them, pairs of 16..127 feed them
+                float mc[8];
 #pragma unroll
-                for (int c = 4; c < kTileN; c += 2) mc[(c >> 1) & 3] = max3(mc[(c >> 1) & 3], s[c], s[c + 1]);
-                m_blk = max3(mc[0], mc[1], fmaxf(mc[2], mc[3]));
+                for (int h = 0; h < 8; ++h) mc[h] = fmaxf(s[2 * h], s[2 * h + 1]);
+#pragma unroll
+                for (int c = 16; c < kTileN; c += 16)
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) mc[h] = max3(mc[h], s[c + 2 * h], s[c + 2 * h + 1]);
+                m_blk = max3(max3(mc[0], mc[1], mc[2]), max3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
                 if constexpr (!kBias) m_blk *= sl2;
+                m_blk += row_off;
             }
 
             const float m_new = fmaxf(m_run, m_blk);
@@ -677,7 +708,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
             // p = 2^(x - shift), two columns per packed FMA / ADD / convert
             float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
             const float mult = kBias ? 1.f : sl2;
-            const float nshift = -shift;
+            const float nshift = row_off - shift;
             uint32_t pk[64];
 #pragma unroll
             for (int c = 0; c < kTileN; c += 4) {

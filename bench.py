@@ -332,11 +332,13 @@ def main():
         fa.fa_fwd(q, k, v, out=out, softmax_max=smax, softmax_sum=ssum, **kw)
 
     torch.cuda.synchronize(dev)
-    t_host = time.perf_counter()
+    host_times = []
     for _ in range(args.warmup):
+        t_host = time.perf_counter()
         flush.zero_()
         step()
-    host_s = (time.perf_counter() - t_host) / args.warmup  # host enqueue time per step
+        host_times.append(time.perf_counter() - t_host)
+    host_s = statistics.median(host_times)  # host enqueue time per step (first-call costs excluded)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if dist:
