@@ -241,15 +241,33 @@ extern "C" fa_status fa_fwd_get_workspace_size(
     if (sink && (!same_shape(sink, {qv.N}) || sink->strides[0] != 1)) return fail(FA_ERR_INNER_NULLPTR);
 
     // position bias
-    if (realShift && pseType == FA_PSE_DENSE) {
-        if (L == L_TND || realShift->ndim != 4) return fail(FA_ERR_INNER_NULLPTR);
+    if (realShift && pseType == FA_PSE_DENSE && L == L_TND) {
+        // [pseTotalLen]: sequence b's [N, Sq_b, Skv_b] block after those of
+        // sequences 0 .. b-1 (aclnnFlashAttentionVarLenScoreV5, realShiftOptional)
+        int64_t total = 0;
+        std::vector<int64_t> offs(B);
+        for (int64_t b = 0; b < B; ++b) {
+            offs[b] = total;
+            total += qv.N * (ex->cu[b + 1] - ex->cu[b]) * (ex->cu[B + 2 + b] - ex->cu[B + 1 + b]);
+        }
+        if (realShift->ndim != 1 || realShift->shape[0] != total || (total > 1 && realShift->strides[0] != 1))
+            return fail(FA_ERR_INNER_NULLPTR);
+        ex->cu.insert(ex->cu.end(), offs.begin(), offs.end());  // copied to the workspace with the offsets
+        p.pse_flat = 1;
+    } else if (realShift && pseType == FA_PSE_DENSE) {
+        if (realShift->ndim != 4) return fail(FA_ERR_INNER_NULLPTR);
         const int64_t* sh = realShift->shape;
-        if (!(sh[0] == 1 || sh[0] == B) || !(sh[1] == 1 || sh[1] == qv.N) || sh[2] != qv.S ||
+        // [B|1, N|1, Sq, Skv], or the compressed [B|1, N|1, 1024, Skv] (the last
+        // 1024 rows of a lower-triangular bias; Sq > 1024, Sq = Skv, keys at or
+        // left of the diagonal only: same page, realShiftOptional notes)
+        const bool rows1024 = sh[2] == 1024 && qv.S > 1024 && qv.S == kv.S && next_c <= 0;
+        if (!(sh[0] == 1 || sh[0] == B) || !(sh[1] == 1 || sh[1] == qv.N) || (sh[2] != qv.S && !rows1024) ||
             sh[3] != kv.S || realShift->strides[3] != 1)
             return fail(FA_ERR_INNER_NULLPTR);
         p.pse_b = sh[0] == 1 ? 0 : realShift->strides[0];
         p.pse_n = sh[1] == 1 ? 0 : realShift->strides[1];
         p.pse_i = realShift->strides[2];
+        p.pse_rows1024 = rows1024 ? 1 : 0;
     } else if (realShift && pseType == FA_PSE_ALIBI) {
         if (same_shape(realShift, {qv.N}) && realShift->strides[0] == 1) {
             p.pse_b = 0; p.pse_n = 1;
@@ -325,6 +343,7 @@ extern "C" fa_status fa_fwd_get_workspace_size(
     p.o_vec32 = aligned32(p.o) && p.o_b % 16 == 0 && p.o_n % 16 == 0 && p.o_s % 16 == 0;
     p.st_vec32 = aligned32(p.smax) && aligned32(p.ssum) && p.st_b % 8 == 0 && p.st_n % 8 == 0 && p.st_s % 8 == 0;
     p.mask_vec = attenMask && aligned16(p.mask) && p.mask_b % 16 == 0 && p.mask_n % 16 == 0 && p.mask_i % 16 == 0;
+    // 16-byte bias loads: the kernels also check each row's start
     p.pse_vec = realShift && pseType == FA_PSE_DENSE && aligned16(p.pse) && p.pse_b % 8 == 0 &&
                 p.pse_n % 8 == 0 && p.pse_i % 8 == 0;
 
@@ -442,6 +461,7 @@ extern "C" fa_status fa_fwd(void* workspace, uint64_t workspaceSize, fa_executor
             return done(FA_ERR_CUDA);
         p.cu_q = reinterpret_cast<const int64_t*>(ws + ex->off_cu);
         p.cu_kv = p.cu_q + (p.B + 1);
+        if (p.pse_flat) p.pse_off = p.cu_q + 2 * (p.B + 1);
     }
     if (!ex->table.empty()) {
         if (cudaMemcpyAsync(ws + ex->off_table, ex->table.data(), ex->table.size() * sizeof(int4),

@@ -58,6 +58,10 @@ struct FaParams {
     int32_t st_vec32;           // the 8 lanes of a statistics row allow 32-byte stores
     int32_t mask_vec;           // mask rows allow 16-byte loads
     int32_t pse_vec;            // dense bias rows allow 16-byte loads
+    // dense bias layouts besides [B|1, N|1, Sq, Skv]:
+    int32_t pse_rows1024;       // [B|1, N|1, 1024, Skv]: the last 1024 rows of the (lower-triangular) bias
+    int32_t pse_flat;           // TND [sum_b N*Sq_b*Skv_b]: each sequence's [N, Sq_b, Skv_b] block in turn
+    const int64_t* pse_off;     // pse_flat: device, element offset of sequence b's block
     int32_t debug_stall;        // failure injection: the MMA warp waits on a barrier never signalled
 
     // Schedule: tickets [0, n_whole) are whole work items; ticket
@@ -76,6 +80,33 @@ struct FaParams {
 
 // fp32 words per row of a partial result
 inline int part_row_words(int d) { return d + 4; }
+
+#ifdef __CUDACC__
+// Dense bias row of query row i (in-sequence index) for (b, n), as a pointer
+// to element [i][0] and the number of readable columns.  The compressed form
+// holds the bias rows Sq-1024 .. Sq-1; a row above them reads compressed row
+// 0 shifted along its diagonal (bias[i][j] = c[0][j + Sq - 1024 - i]), which
+// is the same value for a bias that depends on i - j only.
+template <typename T>
+__device__ __forceinline__ const T* pse_row_ptr(const FaParams& p, int b, int n, int q_len, int kv_len, int i,
+                                                int* cols) {
+    const T* base = static_cast<const T*>(p.pse);
+    if (p.pse_flat) {
+        *cols = kv_len;
+        return base + p.pse_off[b] + (static_cast<int64_t>(n) * q_len + i) * kv_len;
+    }
+    base += b * p.pse_b + n * p.pse_n;
+    if (p.pse_rows1024) {
+        const int first = q_len - 1024;
+        const int r = i >= first ? i - first : 0;
+        const int shift = i >= first ? 0 : first - i;
+        *cols = kv_len - shift;
+        return base + static_cast<int64_t>(r) * p.pse_i + shift;
+    }
+    *cols = kv_len;
+    return base + static_cast<int64_t>(i) * p.pse_i;
+}
+#endif
 
 enum KernelKind { KERNEL_SIMT = 0, KERNEL_SM100 = 1 };
 

@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) fa_fwd_simt_kernel(const FaPar
 
     float slope = 0.f;
     if (p.pse_type == 2) slope = static_cast<const float*>(p.pse)[b * p.pse_b + n * p.pse_n];
-    const T* pse = (p.pse_type == 1) ? static_cast<const T*>(p.pse) + b * p.pse_b + n * p.pse_n : nullptr;
+    int pse_cols = 0;
+    const T* pse = (p.pse_type == 1 && row_ok) ? pse_row_ptr<T>(p, b, n, q_len, kv_len, i, &pse_cols) : nullptr;
     const uint8_t* mask = p.mask_on ? p.mask + b * p.mask_b + n * p.mask_n : nullptr;
 
     float m_run = -CUDART_INF_F, l_lane = 0.f;
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) fa_fwd_simt_kernel(const FaPar
             bool keep = row_ok && j < kv_len && (j - i >= -p.pre) && (j - i <= p.next);
             if (keep && mask) keep = mask[(int64_t)i * p.mask_i + j] == 0;
             float v = x[mm] * p.scale;
-            if (keep && pse) v += to_f(pse[(int64_t)i * p.pse_i + j]);
+            if (keep && pse && j < pse_cols) v += to_f(pse[j]);
             if (p.pse_type == 2) v -= slope * fabsf((float)(i - j));
             x[mm] = keep ? v : -CUDART_INF_F;
             tile_max = fmaxf(tile_max, x[mm]);

@@ -473,6 +473,22 @@ __device__ __forceinline__ void load_bias8(const T* row, int j, int kv_len, bool
     }
 }
 
+// Additive bias of 16 consecutive keys starting at j (times log2(e)): one
+// 32-byte load when the row allows it, else two 8-key loads.
+template <typename T>
+__device__ __forceinline__ void load_bias16(const T* row, int j, int kv_len, bool vec32, bool vec, float* out) {
+    if (vec32 && j + 16 <= kv_len) {
+        uint32_t w[8];
+        ld_global_nc_v8(row + j, w);
+        const T* h = reinterpret_cast<const T*>(w);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) out[e] = to_f(h[e]) * kLog2e;
+    } else {
+        load_bias8(row, j, kv_len, vec, out);
+        load_bias8(row, j + 8, kv_len, vec, out + 8);
+    }
+}
+
 // Excluded flags (nonzero) of 16 consecutive keys starting at j from a mask row.
 __device__ __forceinline__ uint32_t load_mask16(const uint8_t* row, int j, int cols, bool vec) {
     uint32_t bits = 0;
@@ -590,16 +606,29 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
 
         float slope_l2 = 0.f;
         const T* pse_row = nullptr;
+        int pse_cols = 0;
+        bool pse_vec = false, pse_vec32 = false;
         if constexpr (kBias == 2)
             slope_l2 = static_cast<const float*>(p.pse)[it.b * p.pse_b + it.n * p.pse_n] * kLog2e;
         if constexpr (kBias == 1)
-            if (row_ok)
-                pse_row = static_cast<const T*>(p.pse) + it.b * p.pse_b + it.n * p.pse_n + (int64_t)i * p.pse_i;
+            if (row_ok) {
+                pse_row = pse_row_ptr<T>(p, it.b, it.n, it.q_len, it.kv_len, i, &pse_cols);
+                pse_vec = p.pse_vec && (reinterpret_cast<uintptr_t>(pse_row) & 15u) == 0;
+                pse_vec32 = p.pse_vec && (reinterpret_cast<uintptr_t>(pse_row) & 31u) == 0;
+            }
         const uint8_t* mask_row =
             (p.mask_on && row_ok) ? p.mask + it.b * p.mask_b + it.n * p.mask_n + (int64_t)i * p.mask_i : nullptr;
 
         float m_run = -CUDART_INF_F, m_used = -CUDART_INF_F, l = 0.f;
         for (int jb = tr.lo; jb <= tr.hi; ++jb) {
+            if constexpr (kBias == 1) {
+                // the next block's bias row segment (256 bytes) on its way to L2
+                const int jn = (jb + 1) * kTileN;
+                if (pse_row && jb < tr.hi && jn < pse_cols) {
+                    prefetch_l2(pse_row + jn);
+                    if (jn + 64 < pse_cols) prefetch_l2(pse_row + jn + 64);
+                }
+            }
             if (!warp_wait(&bars.s_full[t], s_cnt & 1, abort, kSiteSFull)) { ok = false; break; }
             ++s_cnt;
             tc_fence_after();
@@ -645,19 +674,19 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
             if (kBias && !linear) {
                 const float fi = (float)(i - j0);
 #pragma unroll
-                for (int c8 = 0; c8 < kTileN; c8 += 8) {
-                    float bias[8];
+                for (int c16 = 0; c16 < kTileN; c16 += 16) {
+                    float bias[16];
                     if constexpr (kBias == 2) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) bias[e] = -slope_l2 * fabsf(fi - (float)(c8 + e));
+                        for (int e = 0; e < 16; ++e) bias[e] = -slope_l2 * fabsf(fi - (float)(c16 + e));
                     } else if (pse_row) {
-                        load_bias8(pse_row, j0 + c8, it.kv_len, p.pse_vec != 0, bias);
+                        load_bias16(pse_row, j0 + c16, pse_cols, pse_vec32, pse_vec, bias);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) bias[e] = 0.f;
+                        for (int e = 0; e < 16; ++e) bias[e] = 0.f;
                     }
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) s[c8 + e] = fmaf(s[c8 + e], sl2, bias[e]);
+                    for (int e = 0; e < 16; ++e) s[c16 + e] = fmaf(s[c16 + e], sl2, bias[e]);
                 }
             }
             if (!full) {

@@ -186,6 +186,19 @@ def kernels_per_call(fa, q, k, v, kw):
     return 1 + (1 if pieces > 0 else 0)
 
 
+def alibi_bias_on_device(slopes, seq, first_row, dtype, dev):
+    """Materialised ALiBi bias -slope_n * |i - j| as a dense [1, N, seq - first_row, seq]
+    tensor (rows first_row .. seq-1), built on the device 1024 rows at a time."""
+    n = slopes.shape[0]
+    bias = torch.empty(1, n, seq - first_row, seq, dtype=dtype, device=dev)
+    j = torch.arange(seq, device=dev, dtype=torch.float32)[None, :]
+    for h in range(n):
+        for r0 in range(first_row, seq, 1024):
+            i = torch.arange(r0, min(seq, r0 + 1024), device=dev, dtype=torch.float32)[:, None]
+            bias[0, h, r0 - first_row:r0 - first_row + i.shape[0]] = (-float(slopes[h]) * (i - j).abs()).to(dtype)
+    return bias
+
+
 def fa_kwargs(w, dev):
     c = lambda t: None if t is None else t.to(dev)  # noqa: E731
     pse = c(w.pse)
@@ -254,6 +267,21 @@ def max_over_ranks(values, dist, device):
     return [float(x) for x in t]
 
 
+def hbm_line(bias_bytes, q, k, v, out, ms_per_step):
+    """The materialised-bias band is HBM-heavy: algorithmic bytes (Q, K, V read,
+    O written, and the bias blocks inside the band) per step time, against the
+    measured copy bandwidth."""
+    try:
+        with open(PEAKS_FILE) as f:
+            hbm_peak, src = float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except (OSError, KeyError, ValueError):
+        hbm_peak, src = 6650.0, "fallback 6.65 TB/s"
+    algo = bias_bytes + sum(t.numel() * t.element_size() for t in (q, k, v, out))
+    gbs = algo / (ms_per_step * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+            "algorithmic_bytes": algo, "peak_source": src}
+
+
 def whole_job_tflops(flops_per_rank, world, ms_per_step):
     """Units all ranks processed per step over the slowest rank's step time."""
     return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
@@ -299,6 +327,8 @@ def main():
     ap.add_argument("--workload", type=int, default=2)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--pse", default="slopes", choices=["slopes", "dense", "compressed"],
+                    help="ALiBi workloads: slopes in-kernel, a materialised [1,N,S,S] bias, or its last 1024 rows")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -323,6 +353,17 @@ def main():
     flops_tiles, flops_exact = tile_flops(w)
     q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
     kw = fa_kwargs(w, dev)
+    bias_bytes = 0
+    if args.pse != "slopes" and w.pse_type == 2:
+        # the same ALiBi bias, materialised in the query dtype and resident in HBM
+        # (a fixed positional table, not a per-step input)
+        seq = w.q.shape[1] if w.layout in ("BSH", "BSND") else w.q.shape[2]
+        first = 0 if args.pse == "dense" else seq - 1024
+        kw["real_shift"] = alibi_bias_on_device(w.pse.double().numpy(), seq, first, q.dtype, dev)
+        kw["pse_type"] = 1
+        # bias bytes the kernel reads: one 128x128 block per counted tile-block
+        d = w.q.shape[-1] // w.head_num if w.layout in ("BSH", "SBH") else w.q.shape[-1]
+        bias_bytes = flops_tiles / (4.0 * d) * q.element_size()
     out, smax, ssum = fa.fa_fwd(q, k, v, **kw)
     launches_per_step = kernels_per_call(fa, q, k, v, kw)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -403,22 +444,28 @@ def main():
     value = whole_job_tflops(flops_tiles, world, ms_per_step)
     per_gpu = flops_tiles / (ms_per_step * 1e-3) / 1e12
     peak, peak_src = load_peak()
-    traffic = load_traffic(w.name)
+    traffic = load_traffic(w.name) if args.pse == "slopes" else None
     fl, secs, heads = time_oracle(w, args.cpu_budget)
     cpu_value = fl / secs / 1e12
+    desc = workload_desc(w)
+    if args.pse != "slopes" and w.pse_type == 2:
+        desc["pse"] = ("materialised fp16 bias [1,N,S,S], resident" if args.pse == "dense"
+                       else "compressed bias: last 1024 rows [1,N,1024,S], resident")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": dict(workload_desc(w), parallelism=f"dp{world} (independent shards)",
+        "config": dict(desc, parallelism=f"dp{world} (independent shards)",
                        l2=f"flushed before every step (256 MiB write); Q/K/V/O {qkvo_mb:.0f} MB",
                        flops_tile_counted=flops_tiles, flops_exact=flops_exact,
                        pct_of_nominal_2250=100.0 * per_gpu / 2250.0),
         "roofline": {"bound": "tensor", "achieved": per_gpu, "peak": peak, "unit": UNIT,
                      "frac": per_gpu / peak, "traffic": traffic, "peak_source": peak_src},
+        **({"hbm": hbm_line(bias_bytes, q, k, v, out, ms_per_step)} if args.pse == "dense" else {}),
         "cpu_baseline": {"value": cpu_value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                          "sample": f"{heads} whole (batch, head) pairs of the workload, float64 NumPy, "
-                                   f"{secs:.1f} s"},
+                                   f"{secs:.1f} s" + ("" if args.pse == "slopes" else
+                                                      " (bias from the slopes, the same values in float64)")},
         "e2e": {"value": whole_job_tflops(flops_tiles, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": args.steps * launches_per_step,

@@ -153,14 +153,44 @@ def _head_inputs(layout, qh, kh, vh, b, n, n_kv, seq):
     return qh[b, n, :ql, :], kh[b, n_kv, :kl, :], vh[b, n_kv, :kl, :]
 
 
-def _pse_rows(pse, pse_type, b, n, rows, kv_len):
-    """Additive bias rows [len(rows), kv_len] for (b, n), or None."""
+def _pse_rows(pse, pse_type, b, n, rows, kv_len, seqs=None, n_heads=None):
+    """Additive bias rows [len(rows), kv_len] for (b, n), or None.
+
+    Dense bias layouts (aclnnFlashAttentionVarLenScoreV5, realShiftOptional
+    and its notes on alibi compression and TND):
+      [B or 1, N or 1, Sq, Skv]  the bias itself;
+      [B or 1, N or 1, 1024, Skv] with Sq > 1024 (the compressed form): the last
+          1024 rows of the full bias, alibi_compress = pse[:, :, -1024:, :].  A
+          row i above them is read along its diagonal from the first stored
+          row: bias[i][j] = stored[0][j + (Sq - 1024 - i)] (reading: for a bias
+          that depends on i - j only this is the full bias; columns past the
+          stored row, which the lower-triangular mask excludes, read 0);
+      [sum_b N * Sq_b * Skv_b] (TND): sequence b's [N, Sq_b, Skv_b] block,
+          flattened, after the blocks of sequences 0 .. b-1.
+    """
     if pse is None or pse_type in (0, None):
         return None
     pse = np.asarray(pse, dtype=np.float64)
-    if pse_type == 1:  # dense tensor [B or 1, N or 1, Sq, Skv]
+    rows = np.asarray(rows)
+    if pse_type == 1 and pse.ndim == 1:
+        off = sum(n_heads * s[1] * s[3] for s in seqs[:b])
+        q_len = seqs[b][1]
+        block = pse[off:off + n_heads * q_len * kv_len].reshape(n_heads, q_len, kv_len)
+        return block[n][rows]
+    if pse_type == 1:  # dense tensor [B or 1, N or 1, Sq or 1024, Skv]
         bb = b if pse.shape[0] > 1 else 0
         nn = n if pse.shape[1] > 1 else 0
+        q_len = seqs[b][1] if seqs is not None else pse.shape[2]
+        if pse.shape[2] == 1024 and q_len > 1024:
+            first = q_len - 1024
+            out = np.zeros((len(rows), kv_len))
+            for k, i in enumerate(rows):
+                if i >= first:
+                    out[k] = pse[bb, nn, i - first, :kv_len]
+                else:
+                    shift = first - i
+                    out[k, :kv_len - shift] = pse[bb, nn, 0, shift:kv_len]
+            return out
         return pse[bb, nn][rows][:, :kv_len]
     if pse_type == 2:  # slopes [N] or [B, N]: pse_ij = -slope * |i - j|
         slope = pse[b, n] if pse.ndim == 2 else pse[n]
@@ -219,7 +249,7 @@ def forward(query, key, value, *, layout, head_num, scale, pse=None, pse_type=No
             qs, ks, vs = _head_inputs(layout, qh, kh, vh, b, n, n // group, seq)
             o, m, l = head_forward(
                 qs, ks, vs, scale, rows=rows,
-                pse=_pse_rows(pse, pse_type, b, n, rows, kv_len),
+                pse=_pse_rows(pse, pse_type, b, n, rows, kv_len, seqs, n_q),
                 excluded=_mask_rows(atten_mask, b, n, rows, kv_len),
                 pre_tokens=pre_tokens, next_tokens=next_tokens,
                 sink=None if sink_arr is None else sink_arr[n])
@@ -261,7 +291,7 @@ def forward_rows(query, key, value, rows, *, layout, head_num, scale, pse=None, 
         r = np.array([i])
         o, m, l = head_forward(
             qs[i:i + 1], ks, vs, scale, rows=r,
-            pse=_pse_rows(pse, pse_type, b, n, r, seq[3]),
+            pse=_pse_rows(pse, pse_type, b, n, r, seq[3], seqs, head_num),
             excluded=_mask_rows(atten_mask, b, n, r, seq[3]),
             pre_tokens=pre_tokens, next_tokens=next_tokens,
             sink=None if sink_arr is None else sink_arr[n])

@@ -354,3 +354,38 @@ def test_sink_pse_and_mask_shapes():
     assert plan(q, k, v, atten_mask=torch.zeros(1, 2, 16, 16, dtype=torch.uint8))[0] == 0
     for shape in [(16, 15), (3, 1, 16, 16), (2, 3, 16, 16), (16,)]:
         assert plan(q, k, v, atten_mask=torch.zeros(shape, dtype=torch.bool))[0] == fa.FA_ERR_INNER_NULLPTR, shape
+
+
+# ---------------------------------------------------------------------------
+# Dense bias layouts besides [B|1, N|1, Sq, Skv]
+# ---------------------------------------------------------------------------
+
+def test_plan_compressed_bias_rows():
+    q, k, v = qkv((1, 2, 1100, 64), torch.float16)
+    pse = torch.zeros(1, 2, 1024, 1100, dtype=torch.float16)
+    st, _, _ = plan(q, k, v, real_shift=pse, pse_type=1, next_tokens=0)
+    assert st == 0
+    # only for a lower-triangular band (keys at or left of the diagonal)
+    st, _, _ = plan(q, k, v, real_shift=pse, pse_type=1)
+    assert st == _abi.FA_ERR_INNER_NULLPTR
+    # only when Sq > 1024 and Sq = Skv
+    q2, k2, v2 = qkv((1, 2, 1000, 64), torch.float16)
+    st, _, _ = plan(q2, k2, v2, real_shift=torch.zeros(1, 2, 1024, 1000, dtype=torch.float16), pse_type=1,
+                    next_tokens=0)
+    assert st == _abi.FA_ERR_INNER_NULLPTR
+
+
+def test_plan_tnd_flat_bias_length_and_workspace():
+    lens = [300, 129, 700]
+    cum = [sum(lens[:i + 1]) for i in range(len(lens))]
+    q, k, v = qkv((sum(lens), 2, 128), torch.bfloat16)
+    total = sum(2 * x * x for x in lens)
+    st, ws, _ = plan(q, k, v, input_layout="TND", head_num=2, actual_seq_qlen=cum, actual_seq_kvlen=cum,
+                     real_shift=torch.zeros(total, dtype=torch.bfloat16), pse_type=1)
+    assert st == 0
+    st2, ws0, _ = plan(q, k, v, input_layout="TND", head_num=2, actual_seq_qlen=cum, actual_seq_kvlen=cum)
+    # the per-sequence bias offsets travel with the cumulative lengths
+    assert ws >= ws0 and ws - ws0 <= 256
+    st, _, _ = plan(q, k, v, input_layout="TND", head_num=2, actual_seq_qlen=cum, actual_seq_kvlen=cum,
+                    real_shift=torch.zeros(total - 1, dtype=torch.bfloat16), pse_type=1)
+    assert st == _abi.FA_ERR_INNER_NULLPTR

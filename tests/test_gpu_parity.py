@@ -321,3 +321,59 @@ def test_split_random_mask_with_rows_empty_in_some_pieces():
     w.atten_mask = mask
     assert _split_of(w) == (1, 8)
     compare_full(w)
+
+
+# ---------------------------------------------------------------------------
+# Dense bias layouts besides [B|1, N|1, Sq, Skv]: the compressed last 1024
+# rows of a lower-triangular bias, and the flattened TND bias
+# ---------------------------------------------------------------------------
+
+def _alibi_rows(slopes, sq, skv, first_row, dtype):
+    i = torch.arange(first_row, sq, dtype=torch.float64)[:, None]
+    j = torch.arange(skv, dtype=torch.float64)[None, :]
+    return torch.stack([-s * (i - j).abs() for s in slopes])[None].to(DT[dtype])
+
+
+DT = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
+
+
+@pytest.mark.parametrize("dtype,d", [("f16", 64), ("bf16", 128), ("f32", 64)])
+def test_compressed_alibi_bias(dtype, d):
+    s, n = 1100, 2
+    w = W("BNSD", dtype, (1, n, s, d), n, 3300, next_tokens=0, pre_tokens=600)
+    w.pse = _alibi_rows([0.5, 0.0625], s, s, s - 1024, dtype)  # [1, N, 1024, S]
+    w.pse_type = 1
+    compare_full(w)
+
+
+def test_compressed_bias_not_translation_invariant():
+    # arbitrary stored values: the kernel must read them as the oracle's reading says
+    s, n = 1090, 2
+    w = W("BSND", "bf16", (2, s, n, 128), n, 3310, next_tokens=0)
+    w.pse = normal((2, n, 1024, s), "bf16", 3315)
+    w.pse_type = 1
+    compare_full(w)
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f16", 64), ("f32", 128)])
+def test_tnd_flat_bias(dtype, d):
+    lq, lk, n = [300, 129, 700], [260, 400, 700], 2
+    w = W("TND", dtype, (sum(lq), n, d), n, 3400, kshape=(sum(lk), n, d),
+          actual_seq_q=cumulative(lq, False), actual_seq_kv=cumulative(lk, False))
+    w.pse = torch.cat([normal((n, a, b), dtype, 3405 + i).reshape(-1) for i, (a, b) in enumerate(zip(lq, lk))])
+    w.pse_type = 1
+    compare_full(w)
+
+
+def test_full_size_band_with_compressed_bias_sampled():
+    # the band + ALiBi workload at full size with the bias given as its last
+    # 1024 rows (the layout `bench.py --workload 5 --pse compressed` times)
+    w = build(5)
+    s = w.q.shape[1]
+    slopes = w.pse.double().tolist()
+    w.pse = _alibi_rows(slopes, s, s, s - 1024, w.dtype)  # [1, 16, 1024, 16384]
+    w.pse_type = 1
+    res = run_gpu(w)
+    for t in res:
+        assert not torch.isnan(t).any()
+    compare_rows(w, res, sample_rows(w, 16, seed=55))

@@ -347,3 +347,69 @@ def test_forward_rows_matches_forward():
         np.testing.assert_allclose(o[r], full["out"][bb, i, nn], rtol=1e-13, atol=1e-15)
         np.testing.assert_allclose(m[r], full["softmax_max"][bb, nn, i, 0], rtol=1e-14)
         np.testing.assert_allclose(l[r], full["softmax_sum"][bb, nn, i, 0], rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Dense bias layouts besides [B|1, N|1, Sq, Skv]
+# (aclnnFlashAttentionVarLenScoreV5, realShiftOptional and its notes).
+# ---------------------------------------------------------------------------
+
+def _alibi_full(slopes, sq, skv):
+    i = np.arange(sq, dtype=np.float64)[:, None]
+    j = np.arange(skv, dtype=np.float64)[None, :]
+    return np.stack([-s * np.abs(i - j) for s in slopes])[None]  # [1, N, Sq, Skv]
+
+
+@pytest.mark.parametrize("nxt", [0, -3])
+def test_compressed_alibi_bias_equals_slopes(nxt):
+    # The last 1024 rows of an ALiBi bias (alibi_compress = pse[:, :, -1024:, :])
+    # under a lower-triangular band reproduce the slope-generated bias, which
+    # the oracle computes from -slope * |i - j| on its own path (pse type 2).
+    s, n, d = 1100, 2, 8
+    q, k, v = rand((1, n, s, d), 901), rand((1, n, s, d), 902), rand((1, n, s, d), 903)
+    slopes = np.array([0.5, 0.03125])
+    full = _alibi_full(slopes, s, s)
+    kw = dict(layout="BNSD", head_num=n, scale=d ** -0.5, pre_tokens=300, next_tokens=nxt)
+    want = ref.forward(q, k, v, pse=slopes, pse_type=2, **kw)
+    got_full = ref.forward(q, k, v, pse=full, pse_type=1, **kw)
+    got_c = ref.forward(q, k, v, pse=full[:, :, -1024:, :].copy(), pse_type=1, **kw)
+    for got in (got_full, got_c):
+        np.testing.assert_allclose(got["out"], want["out"], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(got["softmax_max"], want["softmax_max"], rtol=1e-13)
+        np.testing.assert_allclose(got["softmax_sum"], want["softmax_sum"], rtol=1e-12)
+
+
+def test_compressed_bias_rows_are_read_along_the_diagonal():
+    # a bias that is not a function of i - j tells apart which stored entry
+    # each full-bias position reads: rows at or below Sq - 1024 read their own
+    # stored row; a row above reads stored row 0 shifted by (Sq - 1024 - i)
+    s, n = 1030, 1
+    stored = rand((1, n, 1024, s), 904)
+    rows = np.array([0, 3, 5, 6, 700, 1029])
+    got = ref._pse_rows(stored, 1, 0, 0, rows, s, seqs=[(0, s, 0, s)], n_heads=n)
+    first = s - 1024
+    for r_, i in enumerate(rows):
+        for j in (0, 1, i - 1, i):
+            if j < 0:
+                continue
+            want = stored[0, 0, i - first, j] if i >= first else stored[0, 0, 0, j + first - i]
+            assert got[r_, j] == want
+
+
+def test_tnd_flat_bias_equals_each_sequence_with_its_own_bias():
+    lq, lk, n, d = [5, 9, 3], [7, 4, 6], 2, 8
+    q = rand((sum(lq), n, d), 911)
+    k = rand((sum(lk), n, d), 912)
+    v = rand((sum(lk), n, d), 913)
+    blocks = [rand((n, a, b), 914 + i) for i, (a, b) in enumerate(zip(lq, lk))]
+    flat = np.concatenate([x.reshape(-1) for x in blocks])
+    res = ref.forward(q, k, v, layout="TND", head_num=n, scale=0.3, pse=flat, pse_type=1,
+                      actual_seq_q=cumulative(lq, False), actual_seq_kv=cumulative(lk, False))
+    cq, ck = [0] + cumulative(lq, False), [0] + cumulative(lk, False)
+    for b in range(len(lq)):
+        one = ref.forward(q[None, cq[b]:cq[b + 1]].transpose(0, 2, 1, 3), k[None, ck[b]:ck[b + 1]].transpose(0, 2, 1, 3),
+                          v[None, ck[b]:ck[b + 1]].transpose(0, 2, 1, 3), layout="BNSD", head_num=n, scale=0.3,
+                          pse=blocks[b][None], pse_type=1)
+        np.testing.assert_allclose(res["out"][cq[b]:cq[b + 1]], one["out"][0].transpose(1, 0, 2), atol=1e-13)
+        np.testing.assert_allclose(res["softmax_max"][:, cq[b]:cq[b + 1], 0], one["softmax_max"][0, :, :, 0],
+                                   rtol=1e-13)

@@ -39,6 +39,12 @@ MUTATIONS = [
      "qs, ks, vs = _head_inputs(layout, qh, kh, vh, b, n, n % n_kv, seq)"),
     ("query row index off by one", "rows = np.arange(q_len)", "rows = np.arange(1, q_len + 1)"),
     ("stats in log2 units", "m[r0:r1] = mi", "m[r0:r1] = mi / np.log(2.0)"),
+    ("compressed bias row shift off by one", "out[k, :kv_len - shift] = pse[bb, nn, 0, shift:kv_len]",
+     "out[k, :kv_len - shift - 1] = pse[bb, nn, 0, shift + 1:kv_len]"),
+    ("compressed bias read from the first full rows", "out[k] = pse[bb, nn, i - first, :kv_len]",
+     "out[k] = pse[bb, nn, min(i, 1023), :kv_len]"),
+    ("flat bias sequence offset skips the heads", "off = sum(n_heads * s[1] * s[3] for s in seqs[:b])",
+     "off = sum(s[1] * s[3] for s in seqs[:b])"),
 ]
 
 
@@ -71,6 +77,10 @@ def _run_pins():
     pins.test_varlen_equals_each_sequence_alone()
     pins.test_gqa_equals_repeated_kv_heads()
     pins.test_mask_tensor_broadcast_forms_agree()
+    for nxt in (0, -3):
+        pins.test_compressed_alibi_bias_equals_slopes(nxt)
+    pins.test_compressed_bias_rows_are_read_along_the_diagonal()
+    pins.test_tnd_flat_bias_equals_each_sequence_with_its_own_bias()
 
 
 def _with_ref(mod):
