@@ -84,23 +84,35 @@ def _out_shapes(query, layout, head_num, dv, softmax_out_layout):
 
 def _stage1(query, key, value, out, smax, ssum, *, input_layout, head_num, scale, real_shift,
             pse_type, atten_mask, mask_mode, sink, actual_seq_qlen, actual_seq_kvlen,
-            pre_tokens, next_tokens, keep_prob, inner_precise, softmax_out_layout):
+            pre_tokens, next_tokens, keep_prob, inner_precise, softmax_out_layout,
+            q_start_idx=None, kv_start_idx=None):
     lib = _abi.load()
     tq, tk, tv = _ft(query), _ft(key), _ft(value)
     tpse, tmask, tsink = _ft(real_shift), _ft(atten_mask), _ft(sink)
     to, tmax, tsum = _ft(out), _ft(smax), _ft(ssum)
     aq, nq = _i64_array(actual_seq_qlen)
     akv, nkv = _i64_array(actual_seq_kvlen)
+    qst, nqst = _i64_array(_as_list(q_start_idx))
+    kvst, nkvst = _i64_array(_as_list(kv_start_idx))
     ws = ctypes.c_uint64(0)
     ex = ctypes.c_void_p(None)
-    status = lib.fa_fwd_get_workspace_size(
+    status = lib.fa_fwd_get_workspace_size_v5(
         _ptr(tq), _ptr(tk), _ptr(tv), _ptr(tpse), _ptr(tmask), _ptr(tsink),
-        aq, nq, akv, nkv,
+        aq, nq, akv, nkv, qst, nqst, kvst, nkvst,
         float(scale), float(keep_prob), int(pre_tokens), int(next_tokens),
         int(head_num), input_layout.encode(), int(inner_precise),
         int(mask_mode), int(pse_type), softmax_out_layout.encode(),
         _ptr(tmax), _ptr(tsum), _ptr(to), ctypes.byref(ws), ctypes.byref(ex))
     return status, ws.value, ex
+
+
+def _as_list(x):
+    """None, one int, or a sequence of ints -> None or a list."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return [x]
+    return [int(v) for v in x]
 
 
 def _defaults(query, key, value, input_layout, head_num, scale, real_shift, pse_type):
@@ -115,12 +127,14 @@ def _defaults(query, key, value, input_layout, head_num, scale, real_shift, pse_
 def fa_fwd(query, key, value, *, input_layout, head_num, scale=None, real_shift=None, pse_type=None,
            atten_mask=None, mask_mode=FA_MASK_TENSOR, sink=None, actual_seq_qlen=None,
            actual_seq_kvlen=None, pre_tokens=INT64_MAX, next_tokens=INT64_MAX, keep_prob=1.0,
-           inner_precise=0, softmax_out_layout="", out=None, softmax_max=None, softmax_sum=None):
+           inner_precise=0, softmax_out_layout="", out=None, softmax_max=None, softmax_sum=None,
+           q_start_idx=None, kv_start_idx=None):
     """The operator: returns (attention_out, softmax_max, softmax_sum).
 
-    Arguments mirror fa_fwd_get_workspace_size (include/fa_fwd.h).  Tensors
+    Arguments mirror fa_fwd_get_workspace_size_v5 (include/fa_fwd.h).  Tensors
     must be CUDA tensors on one device; actual_seq_* are host sequences of
-    cumulative lengths without a leading zero.  The work is enqueued on the
+    cumulative lengths without a leading zero; q_start_idx / kv_start_idx are
+    None, one int or one int per sequence.  The work is enqueued on the
     current stream of the query's device.
     """
     if not query.is_cuda:
@@ -139,9 +153,10 @@ def fa_fwd(query, key, value, *, input_layout, head_num, scale=None, real_shift=
         head_num=head_num, scale=scale, real_shift=real_shift, pse_type=pse_type,
         atten_mask=atten_mask, mask_mode=mask_mode, sink=sink, actual_seq_qlen=actual_seq_qlen,
         actual_seq_kvlen=actual_seq_kvlen, pre_tokens=pre_tokens, next_tokens=next_tokens,
-        keep_prob=keep_prob, inner_precise=inner_precise, softmax_out_layout=softmax_out_layout)
+        keep_prob=keep_prob, inner_precise=inner_precise, softmax_out_layout=softmax_out_layout,
+        q_start_idx=q_start_idx, kv_start_idx=kv_start_idx)
     if status != FA_SUCCESS:
-        raise FaError(status, "fa_fwd_get_workspace_size")
+        raise FaError(status, "fa_fwd_get_workspace_size_v5")
     ws = torch.empty(max(1, ws_bytes), dtype=torch.uint8, device=dev) if ws_bytes else None
     stream = torch.cuda.current_stream(dev).cuda_stream
     status = _abi.load().fa_fwd(ctypes.c_void_p(ws.data_ptr() if ws is not None else None),
@@ -154,7 +169,8 @@ def fa_fwd(query, key, value, *, input_layout, head_num, scale=None, real_shift=
 def plan(query, key, value, *, input_layout, head_num, scale=None, real_shift=None, pse_type=None,
          atten_mask=None, mask_mode=FA_MASK_TENSOR, sink=None, actual_seq_qlen=None,
          actual_seq_kvlen=None, pre_tokens=INT64_MAX, next_tokens=INT64_MAX, keep_prob=1.0,
-         inner_precise=0, softmax_out_layout="", out=None, softmax_max=None, softmax_sum=None):
+         inner_precise=0, softmax_out_layout="", out=None, softmax_max=None, softmax_sum=None,
+         q_start_idx=None, kv_start_idx=None):
     """Stage 1 only (no device work): returns (status, workspace_bytes, plan_text)."""
     _, dv, scale, pse_type = _defaults(query, key, value, input_layout, head_num, scale, real_shift, pse_type)
     out_shape, stats_shape = _out_shapes(query, input_layout, head_num, dv, softmax_out_layout)
@@ -170,13 +186,43 @@ def plan(query, key, value, *, input_layout, head_num, scale=None, real_shift=No
         head_num=head_num, scale=scale, real_shift=real_shift, pse_type=pse_type,
         atten_mask=atten_mask, mask_mode=mask_mode, sink=sink, actual_seq_qlen=actual_seq_qlen,
         actual_seq_kvlen=actual_seq_kvlen, pre_tokens=pre_tokens, next_tokens=next_tokens,
-        keep_prob=keep_prob, inner_precise=inner_precise, softmax_out_layout=softmax_out_layout)
+        keep_prob=keep_prob, inner_precise=inner_precise, softmax_out_layout=softmax_out_layout,
+        q_start_idx=q_start_idx, kv_start_idx=kv_start_idx)
     text = ""
     if status == FA_SUCCESS:
         lib = _abi.load()
         text = lib.fa_executor_describe(ex).decode()
         lib.fa_executor_destroy(ex)
     return status, ws_bytes, text
+
+
+def lse_merge(outs, softmax_maxes, softmax_sums, *, input_layout, head_num, sink=None, softmax_out_layout="",
+              actual_seq_qlen=None, out=None, softmax_max=None, softmax_sum=None):
+    """Combine fa_fwd results of the same queries over disjoint key sets
+    (computed without a sink) into the result over their union, adding `sink`
+    once (fa_lse_merge in include/fa_fwd.h).  Returns (out, softmax_max, softmax_sum)."""
+    if not outs or not outs[0].is_cuda:
+        raise ValueError("lse_merge runs on CUDA tensors only (no CPU path)")
+    dev = outs[0].device
+    out = torch.empty_like(outs[0]) if out is None else out
+    softmax_max = torch.empty_like(softmax_maxes[0]) if softmax_max is None else softmax_max
+    softmax_sum = torch.empty_like(softmax_sums[0]) if softmax_sum is None else softmax_sum
+    lib = _abi.load()
+    n = len(outs)
+    t_outs = [_ft(t) for t in outs]
+    t_max = [_ft(t) for t in softmax_maxes]
+    t_sum = [_ft(t) for t in softmax_sums]
+    P = ctypes.POINTER(_abi.FaTensor)
+    arr = lambda ts: (P * n)(*[ctypes.pointer(t) for t in ts])  # noqa: E731
+    aq, nq = _i64_array(actual_seq_qlen)
+    tsink, to, tmax, tsum = _ft(sink), _ft(out), _ft(softmax_max), _ft(softmax_sum)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    status = lib.fa_lse_merge(arr(t_outs), arr(t_max), arr(t_sum), n, _ptr(tsink), int(head_num),
+                              input_layout.encode(), softmax_out_layout.encode(), aq, nq,
+                              _ptr(to), _ptr(tmax), _ptr(tsum), ctypes.c_void_p(stream))
+    if status != FA_SUCCESS:
+        raise FaError(status, "fa_lse_merge")
+    return out, softmax_max, softmax_sum
 
 
 def attention_forward(query, key, value, attn_mask=None, scale=None, fused=True, head_first=False, **kwargs):

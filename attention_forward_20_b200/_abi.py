@@ -20,7 +20,7 @@ FA_MASK_TENSOR, FA_MASK_BAND = 0, 1
 
 INT64_MAX = 2**63 - 1
 
-EXPORTS = ("fa_fwd_get_workspace_size", "fa_fwd", "fa_executor_destroy",
+EXPORTS = ("fa_fwd_get_workspace_size", "fa_fwd_get_workspace_size_v5", "fa_lse_merge", "fa_fwd", "fa_executor_destroy",
            "fa_executor_describe", "fa_device_error", "fa_status_string", "fa_fwd_varlen_static")
 
 
@@ -65,6 +65,28 @@ def load():
         ctypes.c_int64, ctypes.c_int64, ctypes.c_char_p,        # maskMode, pseType, softmaxOutLayout
         P(FaTensor), P(FaTensor), P(FaTensor),                  # softmaxMax, softmaxSum, attentionOut
         P(ctypes.c_uint64), P(ctypes.c_void_p),                 # workspaceSize, executor
+    ]
+    lib.fa_fwd_get_workspace_size_v5.restype = ctypes.c_int32
+    lib.fa_fwd_get_workspace_size_v5.argtypes = [
+        P(FaTensor), P(FaTensor), P(FaTensor),                  # query, key, value
+        P(FaTensor), P(FaTensor), P(FaTensor),                  # realShift, attenMask, sink
+        P(ctypes.c_int64), ctypes.c_int64,                      # actualSeqQLen, nSeqQ
+        P(ctypes.c_int64), ctypes.c_int64,                      # actualSeqKvLen, nSeqKv
+        P(ctypes.c_int64), ctypes.c_int64,                      # qStartIdx, nQStartIdx
+        P(ctypes.c_int64), ctypes.c_int64,                      # kvStartIdx, nKvStartIdx
+        ctypes.c_double, ctypes.c_double, ctypes.c_int64, ctypes.c_int64,  # scale, keepProb, pre, next
+        ctypes.c_int64, ctypes.c_char_p, ctypes.c_int64,        # headNum, inputLayout, innerPrecise
+        ctypes.c_int64, ctypes.c_int64, ctypes.c_char_p,        # maskMode, pseType, softmaxOutLayout
+        P(FaTensor), P(FaTensor), P(FaTensor),                  # softmaxMax, softmaxSum, attentionOut
+        P(ctypes.c_uint64), P(ctypes.c_void_p),                 # workspaceSize, executor
+    ]
+    lib.fa_lse_merge.restype = ctypes.c_int32
+    lib.fa_lse_merge.argtypes = [
+        P(P(FaTensor)), P(P(FaTensor)), P(P(FaTensor)), ctypes.c_int64,  # outs, maxes, sums, count
+        P(FaTensor), ctypes.c_int64, ctypes.c_char_p, ctypes.c_char_p,   # sink, headNum, inputLayout, statsLayout
+        P(ctypes.c_int64), ctypes.c_int64,                               # actualSeqQLen, nSeq
+        P(FaTensor), P(FaTensor), P(FaTensor),                           # attentionOut, softmaxMax, softmaxSum
+        ctypes.c_void_p,                                                 # stream
     ]
     lib.fa_fwd.restype = ctypes.c_int32
     lib.fa_fwd.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]

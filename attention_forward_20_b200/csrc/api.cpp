@@ -98,8 +98,6 @@ bool same_shape(const fa_tensor* t, std::initializer_list<int64_t> dims) {
 
 int64_t clamp64(int64_t x, int64_t lo, int64_t hi) { return x < lo ? lo : (x > hi ? hi : x); }
 
-// Number of 128-key blocks that 128-row query tile [r0, r0+128) touches,
-// for the LPT ordering of the varlen work table.
 // 128-key blocks of the union of the two tiles' key ranges of the query block
 // starting at row r0 (0 when neither tile has a key).
 int64_t union_blocks(int64_t r0, int64_t q_len, int64_t kv_len, int64_t pre, int64_t next) {
@@ -111,6 +109,8 @@ int64_t union_blocks(int64_t r0, int64_t q_len, int64_t kv_len, int64_t pre, int
     return hi / kKvBlock - lo / kKvBlock + 1;
 }
 
+// Number of 128-key blocks that 128-row query tile [r0, r0+128) touches,
+// for the LPT ordering of the varlen work table.
 int64_t kv_blocks_for_tile(int64_t r0, int64_t q_len, int64_t kv_len, int64_t pre, int64_t next) {
     const int64_t r1 = std::min(q_len, r0 + 128) - 1;
     if (r1 < r0 || kv_len <= 0) return 0;
@@ -122,11 +122,13 @@ int64_t kv_blocks_for_tile(int64_t r0, int64_t q_len, int64_t kv_len, int64_t pr
 
 }  // namespace
 
-extern "C" fa_status fa_fwd_get_workspace_size(
+extern "C" fa_status fa_fwd_get_workspace_size_v5(
     const fa_tensor* query, const fa_tensor* key, const fa_tensor* value,
     const fa_tensor* realShift, const fa_tensor* attenMask, const fa_tensor* sink,
     const int64_t* actualSeqQLen, int64_t nSeqQ,
     const int64_t* actualSeqKvLen, int64_t nSeqKv,
+    const int64_t* qStartIdx, int64_t nQStartIdx,
+    const int64_t* kvStartIdx, int64_t nKvStartIdx,
     double scaleValue, double keepProb, int64_t preTokens, int64_t nextTokens,
     int64_t headNum, const char* inputLayout, int64_t innerPrecise,
     int64_t maskMode, int64_t pseType, const char* softmaxOutLayout,
@@ -233,9 +235,36 @@ extern "C" fa_status fa_fwd_get_workspace_size(
 
     // band: -pre <= j - i <= next; the two bounds must intersect
     const int64_t lim = max_q + max_kv + 1;
-    const int64_t pre_c = clamp64(preTokens, -lim, lim);
-    const int64_t next_c = clamp64(nextTokens, -lim, lim);
-    if (pre_c + next_c < 0) return fail(FA_ERR_INNER_NULLPTR);
+    if (clamp64(preTokens, -lim, lim) + clamp64(nextTokens, -lim, lim) < 0) return fail(FA_ERR_INNER_NULLPTR);
+    // Global positions (qStartIdx / kvStartIdx, one value or one per sequence):
+    // the band and ALiBi see qStart + i and kvStart + j, i.e. j - i shifted by
+    // delta = kvStart - qStart, the same for every sequence of the call.
+    int64_t delta = 0;
+    {
+        const int64_t nseq = (L == L_TND) ? B : 1;
+        auto start_at = [&](const int64_t* a, int64_t n, int64_t b, int64_t* v) {
+            if (!a || n == 0) { *v = 0; return true; }
+            if (n == 1) { *v = a[0]; return true; }
+            if (n != nseq) return false;
+            *v = a[b];
+            return true;
+        };
+        for (int64_t b = 0; b < nseq; ++b) {
+            int64_t qs, ks;
+            if (!start_at(qStartIdx, nQStartIdx, b, &qs) || !start_at(kvStartIdx, nKvStartIdx, b, &ks) || qs < 0 ||
+                ks < 0 || qs > kMaxS * 64 || ks > kMaxS * 64)
+                return fail(FA_ERR_INNER_NULLPTR);
+            if (b == 0) delta = ks - qs;
+            else if (ks - qs != delta) return fail(FA_ERR_INNER_NULLPTR);
+        }
+    }
+    // -pre <= (j + delta) - i <= next  <=>  -(pre + delta) <= j - i <= next - delta
+    auto shifted = [&](int64_t bound, int64_t d) {
+        return bound >= lim ? lim : clamp64(clamp64(bound, -lim, lim) + d, -lim, lim);
+    };
+    const int64_t pre_c = shifted(preTokens, delta);
+    const int64_t next_c = shifted(nextTokens, -delta);
+    p.alibi_delta = (int32_t)delta;
 
     // sink
     if (sink && (!same_shape(sink, {qv.N}) || sink->strides[0] != 1)) return fail(FA_ERR_INNER_NULLPTR);
@@ -444,6 +473,23 @@ extern "C" fa_status fa_fwd_get_workspace_size(
     return FA_SUCCESS;
 }
 
+extern "C" fa_status fa_fwd_get_workspace_size(
+    const fa_tensor* query, const fa_tensor* key, const fa_tensor* value,
+    const fa_tensor* realShift, const fa_tensor* attenMask, const fa_tensor* sink,
+    const int64_t* actualSeqQLen, int64_t nSeqQ,
+    const int64_t* actualSeqKvLen, int64_t nSeqKv,
+    double scaleValue, double keepProb, int64_t preTokens, int64_t nextTokens,
+    int64_t headNum, const char* inputLayout, int64_t innerPrecise,
+    int64_t maskMode, int64_t pseType, const char* softmaxOutLayout,
+    const fa_tensor* softmaxMax, const fa_tensor* softmaxSum, const fa_tensor* attentionOut,
+    uint64_t* workspaceSize, fa_executor** executor) {
+    return fa_fwd_get_workspace_size_v5(query, key, value, realShift, attenMask, sink, actualSeqQLen, nSeqQ,
+                                        actualSeqKvLen, nSeqKv, nullptr, 0, nullptr, 0, scaleValue, keepProb,
+                                        preTokens, nextTokens, headNum, inputLayout, innerPrecise, maskMode, pseType,
+                                        softmaxOutLayout, softmaxMax, softmaxSum, attentionOut, workspaceSize,
+                                        executor);
+}
+
 extern "C" fa_status fa_fwd(void* workspace, uint64_t workspaceSize, fa_executor* executor, void* stream) {
     if (!executor) return FA_ERR_PARAM_NULLPTR;
     fa_executor* ex = executor;
@@ -481,6 +527,81 @@ extern "C" fa_status fa_fwd(void* workspace, uint64_t workspaceSize, fa_executor
         err = fa::launch_simt(p, st);
     }
     return done(err == cudaSuccess ? FA_SUCCESS : FA_ERR_CUDA);
+}
+
+extern "C" fa_status fa_lse_merge(const fa_tensor* const* outs, const fa_tensor* const* softmaxMaxes,
+                                  const fa_tensor* const* softmaxSums, int64_t count, const fa_tensor* sink,
+                                  int64_t headNum, const char* inputLayout, const char* softmaxOutLayout,
+                                  const int64_t* actualSeqQLen, int64_t nSeq, const fa_tensor* attentionOut,
+                                  const fa_tensor* softmaxMax, const fa_tensor* softmaxSum, void* stream) {
+    if (!outs || !softmaxMaxes || !softmaxSums || !attentionOut || !softmaxMax || !softmaxSum)
+        return FA_ERR_PARAM_NULLPTR;
+    if (!attentionOut->data || !softmaxMax->data || !softmaxSum->data || (sink && !sink->data))
+        return FA_ERR_PARAM_NULLPTR;
+    if (count < 1 || count > fa::MergeParams::kMax) return FA_ERR_INNER_NULLPTR;
+    for (int64_t k = 0; k < count; ++k)
+        if (!outs[k] || !softmaxMaxes[k] || !softmaxSums[k] || !outs[k]->data || !softmaxMaxes[k]->data ||
+            !softmaxSums[k]->data)
+            return FA_ERR_PARAM_NULLPTR;
+    Layout L;
+    if (!parse_layout(inputLayout, &L)) return FA_ERR_PARAM_INVALID;
+    const char* sol = softmaxOutLayout ? softmaxOutLayout : "";
+    const bool same_as_input = std::strcmp(sol, "same_as_input") == 0;
+    if (!same_as_input && sol[0] != '\0') return FA_ERR_PARAM_INVALID;
+    const int32_t dt = attentionOut->dtype;
+    if (!is_float_dtype(dt) || (sink && sink->dtype != FA_F32)) return FA_ERR_PARAM_INVALID;
+    if (headNum < 1 || headNum > kMaxN) return FA_ERR_INNER_NULLPTR;
+    View ov;
+    if (make_view(attentionOut, L, headNum, 0, &ov) != FA_SUCCESS) return FA_ERR_INNER_NULLPTR;
+    const int64_t B = L == L_TND ? 1 : ov.B;
+    if (L == L_TND && actualSeqQLen && (nSeq < 1 || actualSeqQLen[nSeq - 1] != ov.S)) return FA_ERR_INNER_NULLPTR;
+    if (sink && (!same_shape(sink, {headNum}) || sink->strides[0] != 1)) return FA_ERR_INNER_NULLPTR;
+
+    // statistics strides (b, n, s) of a [.., 8] tensor of this layout
+    auto stat_strides = [&](const fa_tensor* st, int64_t* sb, int64_t* sn, int64_t* ss) {
+        if (st->dtype != FA_F32 || !st->data || st->strides[st->ndim - 1] != 1) return false;
+        if (L != L_TND) {
+            if (!same_shape(st, {ov.B, headNum, ov.S, 8})) return false;
+            *sb = st->strides[0]; *sn = st->strides[1]; *ss = st->strides[2];
+        } else if (same_as_input) {
+            if (!same_shape(st, {ov.S, headNum, 8})) return false;
+            *sb = 0; *ss = st->strides[0]; *sn = st->strides[1];
+        } else {
+            if (!same_shape(st, {headNum, ov.S, 8})) return false;
+            *sb = 0; *sn = st->strides[0]; *ss = st->strides[1];
+        }
+        return true;
+    };
+    fa::MergeParams mp;
+    std::memset(&mp, 0, sizeof(mp));
+    mp.count = (int32_t)count;
+    for (int64_t k = 0; k < count; ++k) {
+        View v;
+        if (outs[k]->dtype != dt || make_view(outs[k], L, headNum, 0, &v) != FA_SUCCESS || v.N != ov.N ||
+            v.S != ov.S || v.D != ov.D || (L != L_TND && v.B != ov.B))
+            return FA_ERR_INNER_NULLPTR;
+        int64_t a, b, c, a2, b2, c2;
+        if (!stat_strides(softmaxMaxes[k], &a, &b, &c) || !stat_strides(softmaxSums[k], &a2, &b2, &c2) ||
+            a != a2 || b != b2 || c != c2)
+            return FA_ERR_INNER_NULLPTR;
+        mp.out[k] = outs[k]->data;
+        mp.smax[k] = static_cast<const float*>(softmaxMaxes[k]->data);
+        mp.ssum[k] = static_cast<const float*>(softmaxSums[k]->data);
+        mp.o_b[k] = v.sb; mp.o_n[k] = v.sn; mp.o_s[k] = v.ss;
+        mp.st_b[k] = a; mp.st_n[k] = b; mp.st_s[k] = c;
+    }
+    int64_t a, b, c, a2, b2, c2;
+    if (!stat_strides(softmaxMax, &a, &b, &c) || !stat_strides(softmaxSum, &a2, &b2, &c2) || a != a2 || b != b2 ||
+        c != c2)
+        return FA_ERR_INNER_NULLPTR;
+    mp.res_o = attentionOut->data;
+    mp.res_max = static_cast<float*>(softmaxMax->data);
+    mp.res_sum = static_cast<float*>(softmaxSum->data);
+    mp.r_o_b = ov.sb; mp.r_o_n = ov.sn; mp.r_o_s = ov.ss;
+    mp.r_st_b = a; mp.r_st_n = b; mp.r_st_s = c;
+    mp.sink = sink ? static_cast<const float*>(sink->data) : nullptr;
+    mp.B = (int32_t)B; mp.N = (int32_t)headNum; mp.S = (int32_t)ov.S; mp.Dv = (int32_t)ov.D; mp.dtype = dt;
+    return fa::launch_lse_merge(mp, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_SUCCESS : FA_ERR_CUDA;
 }
 
 extern "C" void fa_executor_destroy(fa_executor* executor) { delete executor; }

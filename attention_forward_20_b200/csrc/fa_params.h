@@ -62,6 +62,7 @@ struct FaParams {
     int32_t pse_rows1024;       // [B|1, N|1, 1024, Skv]: the last 1024 rows of the (lower-triangular) bias
     int32_t pse_flat;           // TND [sum_b N*Sq_b*Skv_b]: each sequence's [N, Sq_b, Skv_b] block in turn
     const int64_t* pse_off;     // pse_flat: device, element offset of sequence b's block
+    int32_t alibi_delta;        // kvStartIdx - qStartIdx: ALiBi distance |i - j - delta| (global positions)
     int32_t debug_stall;        // failure injection: the MMA warp waits on a barrier never signalled
 
     // Schedule: tickets [0, n_whole) are whole work items; ticket
@@ -107,6 +108,25 @@ __device__ __forceinline__ const T* pse_row_ptr(const FaParams& p, int b, int n,
     return base + static_cast<int64_t>(i) * p.pse_i;
 }
 #endif
+
+// fa_lse_merge: partial results of one query set over disjoint key sets.
+// Rows are addressed as (b, n, s) with element strides (TND: b = 0, s = token).
+struct MergeParams {
+    static constexpr int kMax = 16;
+    int32_t count;
+    const void* out[kMax];
+    const float* smax[kMax];
+    const float* ssum[kMax];
+    int64_t o_b[kMax], o_n[kMax], o_s[kMax];
+    int64_t st_b[kMax], st_n[kMax], st_s[kMax];
+    void* res_o;
+    float* res_max;
+    float* res_sum;
+    int64_t r_o_b, r_o_n, r_o_s, r_st_b, r_st_n, r_st_s;
+    const float* sink;  // fp32 [N] or nullptr
+    int32_t B, N, S, Dv, dtype;
+};
+cudaError_t launch_lse_merge(const MergeParams& mp, cudaStream_t stream);
 
 enum KernelKind { KERNEL_SIMT = 0, KERNEL_SM100 = 1 };
 

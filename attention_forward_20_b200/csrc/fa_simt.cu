@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) fa_fwd_simt_kernel(const FaPar
             if (keep && mask) keep = mask[(int64_t)i * p.mask_i + j] == 0;
             float v = x[mm] * p.scale;
             if (keep && pse && j < pse_cols) v += to_f(pse[j]);
-            if (p.pse_type == 2) v -= slope * fabsf((float)(i - j));
+            if (p.pse_type == 2) v -= slope * fabsf((float)(i - j - p.alibi_delta));
             x[mm] = keep ? v : -CUDART_INF_F;
             tile_max = fmaxf(tile_max, x[mm]);
         }

@@ -651,12 +651,13 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                 // A block wholly on one side of every row's diagonal has
                 // -slope·|i - j| = st·c - st·(i - j0) with st = ±slope: a ramp
                 // over the columns plus a per-row constant.
-                const bool below = j0 + kTileN - 1 <= r0;
-                const bool above = j0 >= r0 + kTileM - 1;
+                const int j0g = j0 + p.alibi_delta;  // key positions relative to the query positions
+                const bool below = j0g + kTileN - 1 <= r0;
+                const bool above = j0g >= r0 + kTileM - 1;
                 linear = below || above;
                 if (linear) {
                     const float st = below ? slope_l2 : -slope_l2;
-                    row_off = -st * (float)(i - j0);
+                    row_off = -st * (float)(i - j0g);
                     float t[8];  // ramp at columns c8 + h, four chains of column pairs
 #pragma unroll
                     for (int h = 0; h < 8; ++h) t[h] = st * (float)h;
@@ -672,7 +673,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                 }
             }
             if (kBias && !linear) {
-                const float fi = (float)(i - j0);
+                const float fi = (float)(i - j0 - p.alibi_delta);
 #pragma unroll
                 for (int c16 = 0; c16 < kTileN; c16 += 16) {
                     float bias[16];

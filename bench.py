@@ -267,7 +267,7 @@ def max_over_ranks(values, dist, device):
     return [float(x) for x in t]
 
 
-def hbm_line(bias_bytes, q, k, v, out, ms_per_step):
+def hbm_line(bias_bytes, q, k, v, out, ms_per_step, bytes_override=None):
     """The materialised-bias band is HBM-heavy: algorithmic bytes (Q, K, V read,
     O written, and the bias blocks inside the band) per step time, against the
     measured copy bandwidth."""
@@ -277,6 +277,8 @@ def hbm_line(bias_bytes, q, k, v, out, ms_per_step):
     except (OSError, KeyError, ValueError):
         hbm_peak, src = 6650.0, "fallback 6.65 TB/s"
     algo = bias_bytes + sum(t.numel() * t.element_size() for t in (q, k, v, out))
+    if bytes_override is not None:
+        algo = bytes_override
     gbs = algo / (ms_per_step * 1e-3) / 1e9
     return {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
             "algorithmic_bytes": algo, "peak_source": src}
@@ -327,6 +329,9 @@ def main():
     ap.add_argument("--workload", type=int, default=2)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--kv-chunks", type=int, default=1,
+                    help="split the keys into this many chunks: one forward per chunk at its kvStartIdx, "
+                         "then fa_lse_merge (dense layouts)")
     ap.add_argument("--pse", default="slopes", choices=["slopes", "dense", "compressed"],
                     help="ALiBi workloads: slopes in-kernel, a materialised [1,N,S,S] bias, or its last 1024 rows")
     args = ap.parse_args()
@@ -366,11 +371,41 @@ def main():
         bias_bytes = flops_tiles / (4.0 * d) * q.element_size()
     out, smax, ssum = fa.fa_fwd(q, k, v, **kw)
     launches_per_step = kernels_per_call(fa, q, k, v, kw)
+    if args.kv_chunks > 1:
+        launches_per_step = args.kv_chunks * launches_per_step + 1  # chunk forwards + the merge (upper bound)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
         fa.fa_fwd(q, k, v, out=out, softmax_max=smax, softmax_sum=ssum, **kw)
+
+    merge_events = []
+    if args.kv_chunks > 1:
+        # a forward split along the keys (as context parallelism would place the
+        # chunks on different GPUs), each chunk at its global start, then the merge
+        seq_axis = {"BNSD": 2, "BSND": 1, "BSH": 1, "SBH": 0}[w.layout]
+        skv = k.shape[seq_axis]
+        bounds = [(c * skv // args.kv_chunks, (c + 1) * skv // args.kv_chunks) for c in range(args.kv_chunks)]
+        kcs = [k.narrow(seq_axis, a, b - a).contiguous() for a, b in bounds]
+        vcs = [v.narrow(seq_axis, a, b - a).contiguous() for a, b in bounds]
+        kw_base = {key_: val for key_, val in kw.items() if key_ != "sink"}
+        mask = kw_base.get("atten_mask")
+        # a chunk's mask is its columns of the mask (masks are indexed by in-chunk positions)
+        kw_parts = [dict(kw_base, atten_mask=None if mask is None else mask[..., a:b].contiguous(), kv_start_idx=a)
+                    for a, b in bounds]
+        parts = [fa.fa_fwd(q, kc, vc, **kp) for kc, vc, kp in zip(kcs, vcs, kw_parts)]
+
+        def step():  # noqa: F811
+            for kc, vc, kp, (po, pm, ps) in zip(kcs, vcs, kw_parts, parts):
+                fa.fa_fwd(q, kc, vc, out=po, softmax_max=pm, softmax_sum=ps, **kp)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fa.lse_merge([p_[0] for p_ in parts], [p_[1] for p_ in parts], [p_[2] for p_ in parts],
+                         input_layout=w.layout, head_num=w.head_num, sink=kw.get("sink"),
+                         softmax_out_layout=w.softmax_out_layout or "", out=out, softmax_max=smax,
+                         softmax_sum=ssum)
+            e1.record(stream)
+            merge_events.append((e0, e1))
 
     torch.cuda.synchronize(dev)
     host_times = []
@@ -448,6 +483,14 @@ def main():
     fl, secs, heads = time_oracle(w, args.cpu_budget)
     cpu_value = fl / secs / 1e12
     desc = workload_desc(w)
+    merge_line = None
+    if args.kv_chunks > 1:
+        desc["kv_chunks"] = f"{args.kv_chunks} key chunks at their kvStartIdx, then fa_lse_merge (sink added there)"
+        timed = merge_events[-args.steps:]
+        merge_ms = sum(a.elapsed_time(b) for a, b in timed) / max(1, len(timed))
+        part_bytes = out.numel() * out.element_size() + 2 * smax.numel() * smax.element_size()
+        merge_line = hbm_line(0, q, k, v, out, merge_ms, bytes_override=(args.kv_chunks + 1) * part_bytes)
+        merge_line["ms"] = merge_ms
     if args.pse != "slopes" and w.pse_type == 2:
         desc["pse"] = ("materialised fp16 bias [1,N,S,S], resident" if args.pse == "dense"
                        else "compressed bias: last 1024 rows [1,N,1024,S], resident")
@@ -462,6 +505,7 @@ def main():
         "roofline": {"bound": "tensor", "achieved": per_gpu, "peak": peak, "unit": UNIT,
                      "frac": per_gpu / peak, "traffic": traffic, "peak_source": peak_src},
         **({"hbm": hbm_line(bias_bytes, q, k, v, out, ms_per_step)} if args.pse == "dense" else {}),
+        **({"merge": merge_line} if merge_line else {}),
         "cpu_baseline": {"value": cpu_value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                          "sample": f"{heads} whole (batch, head) pairs of the workload, float64 NumPy, "
                                    f"{secs:.1f} s" + ("" if args.pse == "slopes" else

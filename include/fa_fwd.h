@@ -107,7 +107,13 @@ typedef struct fa_executor fa_executor;
  *   key/value may have fewer heads than query (Nq % Nkv == 0; query head n
  *   reads key/value head n / (Nq/Nkv)).  value's head dim may be smaller than
  *   the query/key head dim.
- * realShift: optional bias, see FA_PSE_*; NULL for none.
+ * realShift: optional bias, see FA_PSE_*; NULL for none.  A dense bias is
+ *   [B|1, N|1, Sq, Skv]; or its last 1024 rows [B|1, N|1, 1024, Skv] when
+ *   Sq > 1024, Sq == Skv and the band is lower-triangular (nextTokens <= 0):
+ *   row i < Sq-1024 then reads stored row 0 along its diagonal,
+ *   bias[i][j] = stored[0][j + Sq - 1024 - i]; with "TND" it is the 1-D
+ *   [sum_b N*Sq_b*Skv_b], sequence b's [N, Sq_b, Skv_b] block after those of
+ *   sequences 0..b-1 (aclnnFlashAttentionVarLenScoreV5, realShiftOptional).
  * attenMask: optional FA_U8/FA_BOOL, nonzero = excluded.  Shapes [B,N,Sq,Skv],
  *   [B,1,Sq,Skv], [1,1,Sq,Skv] or [Sq,Skv]; with "TND" only [Sq,Skv] indexed by
  *   in-sequence positions (Sq, Skv at least the longest sequence).
@@ -132,13 +138,39 @@ typedef struct fa_executor fa_executor;
  *   memory until fa_fwd() or fa_executor_destroy() releases it.
  *
  * Returns FA_SUCCESS, FA_ERR_PARAM_NULLPTR, FA_ERR_PARAM_INVALID or
- * FA_ERR_INNER_NULLPTR; on error *executor is set to NULL.  Thread-safe; no
- * CUDA call is made. */
+ * FA_ERR_INNER_NULLPTR; on error *executor is set to NULL.  Thread-safe; the
+ * only CUDA calls read the current device's SM count (no device work; with no
+ * device the plan assumes a 148-SM B200). */
 FA_API fa_status fa_fwd_get_workspace_size(
     const fa_tensor* query, const fa_tensor* key, const fa_tensor* value,
     const fa_tensor* realShift, const fa_tensor* attenMask, const fa_tensor* sink,
     const int64_t* actualSeqQLen, int64_t nSeqQ,
     const int64_t* actualSeqKvLen, int64_t nSeqKv,
+    double scaleValue, double keepProb, int64_t preTokens, int64_t nextTokens,
+    int64_t headNum, const char* inputLayout, int64_t innerPrecise,
+    int64_t maskMode, int64_t pseType, const char* softmaxOutLayout,
+    const fa_tensor* softmaxMax, const fa_tensor* softmaxSum, const fa_tensor* attentionOut,
+    uint64_t* workspaceSize, fa_executor** executor);
+
+/* Stage 1 with global positions (aclnnFlashAttentionVarLenScoreV5,
+ * qStartIdxOptional / kvStartIdxOptional: the start, in the whole sequence, of
+ * the query and key/value chunk this call sees).  The band and an ALiBi bias
+ * are evaluated at global positions qStart + i and kvStart + j:
+ *   keep iff -preTokens <= (kvStart + j) - (qStart + i) <= nextTokens,
+ *   ALiBi pse = -slope * |(qStart + i) - (kvStart + j)|;
+ * attenMask and a dense realShift stay indexed by in-chunk positions.
+ * qStartIdx / kvStartIdx: host int64, NULL (0), one value, or one per
+ * sequence (nQStartIdx / nKvStartIdx entries, "TND" only for more than one);
+ * kvStart - qStart must be the same for every sequence (else 561103).  All
+ * other arguments and the return values are those of
+ * fa_fwd_get_workspace_size, which equals this call with both NULL. */
+FA_API fa_status fa_fwd_get_workspace_size_v5(
+    const fa_tensor* query, const fa_tensor* key, const fa_tensor* value,
+    const fa_tensor* realShift, const fa_tensor* attenMask, const fa_tensor* sink,
+    const int64_t* actualSeqQLen, int64_t nSeqQ,
+    const int64_t* actualSeqKvLen, int64_t nSeqKv,
+    const int64_t* qStartIdx, int64_t nQStartIdx,
+    const int64_t* kvStartIdx, int64_t nKvStartIdx,
     double scaleValue, double keepProb, int64_t preTokens, int64_t nextTokens,
     int64_t headNum, const char* inputLayout, int64_t innerPrecise,
     int64_t maskMode, int64_t pseType, const char* softmaxOutLayout,
@@ -154,6 +186,33 @@ FA_API fa_status fa_fwd_get_workspace_size(
  * Returns FA_SUCCESS, FA_ERR_PARAM_NULLPTR (executor NULL, or workspace NULL
  * with a nonzero size), FA_ERR_WORKSPACE or FA_ERR_CUDA. */
 FA_API fa_status fa_fwd(void* workspace, uint64_t workspaceSize, fa_executor* executor, void* stream);
+
+/* Merge of partial results (the step after a forward split along the keys,
+ * e.g. context parallelism: key/value chunks on different GPUs, each run with
+ * its kvStartIdx).  outs[k], softmaxMaxes[k], softmaxSums[k] (k < count,
+ * 1 <= count <= 16) are the attentionOut / softmaxMax / softmaxSum of the same
+ * queries over disjoint key sets, computed without a sink; the result over
+ * the union of the key sets, with the optional sink added once, is
+ *   M   = max(max_k m_k over rows with l_k > 0, sink_n)
+ *   l   = sum_k l_k e^(m_k - M) + e^(sink_n - M)
+ *   out = sum_k l_k e^(m_k - M) out_k / l
+ * (the online-softmax update of the forward formula, applied to whole partial
+ * results; softmaxMax/softmaxSum in natural-log units as the forward writes
+ * them).  A row with no key in any part gets out = 0, m = -inf, l = 0 (with a
+ * sink: m = sink, l = 1).
+ * Tensors are device tensors in `inputLayout` with headNum query heads, all
+ * outs[k] and attentionOut of one dtype and shape; statistics fp32 of the
+ * forward's statistics shape for that layout and softmaxOutLayout.
+ * actualSeqQLen (TND, optional): host cumulative lengths, checked against T.
+ * Enqueued on `stream`; no workspace.  Returns FA_SUCCESS,
+ * FA_ERR_PARAM_NULLPTR, FA_ERR_PARAM_INVALID, FA_ERR_INNER_NULLPTR or
+ * FA_ERR_CUDA.  (No page defines this call; the pages define the statistics
+ * it consumes and name the split scenario that needs it.) */
+FA_API fa_status fa_lse_merge(const fa_tensor* const* outs, const fa_tensor* const* softmaxMaxes,
+                              const fa_tensor* const* softmaxSums, int64_t count, const fa_tensor* sink,
+                              int64_t headNum, const char* inputLayout, const char* softmaxOutLayout,
+                              const int64_t* actualSeqQLen, int64_t nSeq, const fa_tensor* attentionOut,
+                              const fa_tensor* softmaxMax, const fa_tensor* softmaxSum, void* stream);
 
 /* Releases an executor that will not be passed to fa_fwd().  NULL is a no-op. */
 FA_API void fa_executor_destroy(fa_executor* executor);

@@ -84,13 +84,15 @@ def from_heads(o, layout):
 # ---------------------------------------------------------------------------
 
 def head_forward(q, k, v, scale, rows=None, pse=None, excluded=None,
-                 pre_tokens=INT64_MAX, next_tokens=INT64_MAX, sink=None):
+                 pre_tokens=INT64_MAX, next_tokens=INT64_MAX, sink=None, delta=0):
     """Attention of one (batch, head).
 
     q: [R, D] query rows whose in-sequence indices are `rows` (default 0..R-1);
     k: [Skv, D]; v: [Skv, Dv]; pse: [R, Skv] additive bias or None;
     excluded: bool [R, Skv] (True = does not take part) or None;
-    sink: float or None.  Returns o [R, Dv], m [R], l [R] in float64.
+    sink: float or None; delta: kvStartIdx - qStartIdx, the band compares the
+    global positions (kvStart + j) - (qStart + i) = j - i + delta.
+    Returns o [R, Dv], m [R], l [R] in float64.
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -109,7 +111,7 @@ def head_forward(q, k, v, scale, rows=None, pse=None, excluded=None,
         s = scale * (q[r0:r1] @ k.T)
         if pse is not None:
             s = s + np.asarray(pse[r0:r1], dtype=np.float64)
-        diff = j[None, :] - i[:, None]
+        diff = j[None, :] - i[:, None] + delta
         keep = (diff >= -pre_tokens) & (diff <= next_tokens)
         if excluded is not None:
             keep &= ~np.asarray(excluded[r0:r1], dtype=bool)
@@ -153,7 +155,7 @@ def _head_inputs(layout, qh, kh, vh, b, n, n_kv, seq):
     return qh[b, n, :ql, :], kh[b, n_kv, :kl, :], vh[b, n_kv, :kl, :]
 
 
-def _pse_rows(pse, pse_type, b, n, rows, kv_len, seqs=None, n_heads=None):
+def _pse_rows(pse, pse_type, b, n, rows, kv_len, seqs=None, n_heads=None, delta=0):
     """Additive bias rows [len(rows), kv_len] for (b, n), or None.
 
     Dense bias layouts (aclnnFlashAttentionVarLenScoreV5, realShiftOptional
@@ -192,9 +194,9 @@ def _pse_rows(pse, pse_type, b, n, rows, kv_len, seqs=None, n_heads=None):
                     out[k, :kv_len - shift] = pse[bb, nn, 0, shift:kv_len]
             return out
         return pse[bb, nn][rows][:, :kv_len]
-    if pse_type == 2:  # slopes [N] or [B, N]: pse_ij = -slope * |i - j|
+    if pse_type == 2:  # slopes [N] or [B, N]: pse_ij = -slope * |i - j| at global positions
         slope = pse[b, n] if pse.ndim == 2 else pse[n]
-        j = np.arange(kv_len, dtype=np.float64)
+        j = np.arange(kv_len, dtype=np.float64) + delta
         return -slope * np.abs(np.asarray(rows, dtype=np.float64)[:, None] - j[None, :])
     raise ValueError(f"unknown pse_type {pse_type}")
 
@@ -211,9 +213,19 @@ def _mask_rows(mask, b, n, rows, kv_len):
     return mk[bb, nn][rows][:, :kv_len]
 
 
+def _deltas(q_start, kv_start, n_seqs):
+    """kvStartIdx - qStartIdx per sequence (each None, one value or one per sequence)."""
+    def at(x, b):
+        if x is None:
+            return 0
+        x = np.atleast_1d(np.asarray(x, dtype=np.int64))
+        return int(x[0] if x.size == 1 else x[b])
+    return [at(kv_start, b) - at(q_start, b) for b in range(n_seqs)]
+
+
 def forward(query, key, value, *, layout, head_num, scale, pse=None, pse_type=None,
             atten_mask=None, pre_tokens=INT64_MAX, next_tokens=INT64_MAX, sink=None,
-            actual_seq_q=None, actual_seq_kv=None, softmax_out_layout=""):
+            actual_seq_q=None, actual_seq_kv=None, softmax_out_layout="", q_start=None, kv_start=None):
     """Full forward.  Returns dict(out, softmax_max, softmax_sum) in float64.
 
     out has the query layout (value head dim); the statistics are
@@ -228,6 +240,7 @@ def forward(query, key, value, *, layout, head_num, scale, pse=None, pse_type=No
     n_kv = kh.shape[1]
     group = n_q // n_kv
     seqs = _sequences(layout, qh, kh, actual_seq_q, actual_seq_kv)
+    deltas = _deltas(q_start, kv_start, len(seqs))
     dv = vh.shape[-1]
     sink_arr = None if sink is None else np.asarray(sink, dtype=np.float64)
     if layout == "TND":
@@ -249,10 +262,10 @@ def forward(query, key, value, *, layout, head_num, scale, pse=None, pse_type=No
             qs, ks, vs = _head_inputs(layout, qh, kh, vh, b, n, n // group, seq)
             o, m, l = head_forward(
                 qs, ks, vs, scale, rows=rows,
-                pse=_pse_rows(pse, pse_type, b, n, rows, kv_len, seqs, n_q),
+                pse=_pse_rows(pse, pse_type, b, n, rows, kv_len, seqs, n_q, deltas[b]),
                 excluded=_mask_rows(atten_mask, b, n, rows, kv_len),
                 pre_tokens=pre_tokens, next_tokens=next_tokens,
-                sink=None if sink_arr is None else sink_arr[n])
+                sink=None if sink_arr is None else sink_arr[n], delta=deltas[b])
             if layout == "TND":
                 out[seq[0]:seq[0] + q_len, n] = o
                 smax[seq[0]:seq[0] + q_len, n] = m
@@ -272,7 +285,7 @@ def forward(query, key, value, *, layout, head_num, scale, pse=None, pse_type=No
 
 def forward_rows(query, key, value, rows, *, layout, head_num, scale, pse=None, pse_type=None,
                  atten_mask=None, pre_tokens=INT64_MAX, next_tokens=INT64_MAX, sink=None,
-                 actual_seq_q=None, actual_seq_kv=None):
+                 actual_seq_q=None, actual_seq_kv=None, q_start=None, kv_start=None):
     """Selected output rows only: `rows` is a list of (b, n, i), i the in-sequence index.
 
     Returns o [R, Dv], m [R], l [R]; used to check full-size runs row by row.
@@ -283,6 +296,7 @@ def forward_rows(query, key, value, rows, *, layout, head_num, scale, pse=None, 
     vh = heads_view(value, layout, _value_head_dim(value, key, layout, head_dim))
     group = head_num // kh.shape[1]
     seqs = _sequences(layout, qh, kh, actual_seq_q, actual_seq_kv)
+    deltas = _deltas(q_start, kv_start, len(seqs))
     sink_arr = None if sink is None else np.asarray(sink, dtype=np.float64)
     outs, ms, ls = [], [], []
     for (b, n, i) in rows:
@@ -291,14 +305,49 @@ def forward_rows(query, key, value, rows, *, layout, head_num, scale, pse=None, 
         r = np.array([i])
         o, m, l = head_forward(
             qs[i:i + 1], ks, vs, scale, rows=r,
-            pse=_pse_rows(pse, pse_type, b, n, r, seq[3], seqs, head_num),
+            pse=_pse_rows(pse, pse_type, b, n, r, seq[3], seqs, head_num, deltas[b]),
             excluded=_mask_rows(atten_mask, b, n, r, seq[3]),
             pre_tokens=pre_tokens, next_tokens=next_tokens,
-            sink=None if sink_arr is None else sink_arr[n])
+            sink=None if sink_arr is None else sink_arr[n], delta=deltas[b])
         outs.append(o[0])
         ms.append(m[0])
         ls.append(l[0])
     return np.array(outs), np.array(ms), np.array(ls)
+
+
+def merge(outs, maxes, sums, sink=None):
+    """Result over the union of disjoint key sets from per-set results.
+
+    outs[k] [..., Dv], maxes[k] / sums[k] [...]: normalised output, row max
+    and row sum (natural log units) of the same rows over key set k, without
+    a sink.  The forward formula over the union regroups its sums by set:
+    with M the largest max over sets holding a key (and the sink),
+      l = sum_k sums_k e^(maxes_k - M) + e^(sink - M),
+      o = sum_k sums_k e^(maxes_k - M) outs_k / l;
+    rows with no key and no sink give o = 0, m = -inf, l = 0.
+    `sink` broadcasts against the rows (e.g. shape [N, 1] for [N, T] rows).
+    """
+    ms = [np.asarray(x, dtype=np.float64) for x in maxes]
+    ls = [np.asarray(x, dtype=np.float64) for x in sums]
+    os_ = [np.asarray(x, dtype=np.float64) for x in outs]
+    big = np.full(ms[0].shape, -np.inf)
+    for m_k, l_k in zip(ms, ls):
+        big = np.maximum(big, np.where(l_k > 0, m_k, -np.inf))
+    if sink is not None:
+        big = np.maximum(big, np.asarray(sink, dtype=np.float64))
+    shift = np.where(np.isfinite(big), big, 0.0)
+    l = np.zeros(big.shape)
+    o = np.zeros(os_[0].shape)
+    for o_k, m_k, l_k in zip(os_, ms, ls):
+        w = np.where(l_k > 0, l_k * np.exp(np.where(l_k > 0, m_k, 0.0) - shift), 0.0)
+        l = l + w
+        o = o + w[..., None] * o_k
+    if sink is not None:
+        l = l + np.exp(np.asarray(sink, dtype=np.float64) - shift)
+    safe = np.where(l > 0, l, 1.0)
+    o = np.where((l > 0)[..., None], o / safe[..., None], 0.0)
+    m = np.where(l > 0, big, -np.inf)
+    return o, m, l
 
 
 def _head_dim(query, layout, head_num):

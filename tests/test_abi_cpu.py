@@ -1,7 +1,8 @@
 """The C ABI on the CPU: the library loads, exports every function that
 include/fa_fwd.h declares, and stage 1 validates arguments with the status
-codes of the aclnn operator pages (161001 / 161002 / 561103).  Stage 1 makes no
-CUDA call, so host tensors stand in for device ones here."""
+codes of the aclnn operator pages (161001 / 161002 / 561103).  Stage 1 does no
+device work (it only reads the SM count), so host tensors stand in for device
+ones here."""
 import ctypes
 import os
 import re
@@ -26,7 +27,7 @@ def built():
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_header_declares_the_documented_entry_points():
@@ -389,3 +390,42 @@ def test_plan_tnd_flat_bias_length_and_workspace():
     st, _, _ = plan(q, k, v, input_layout="TND", head_num=2, actual_seq_qlen=cum, actual_seq_kvlen=cum,
                     real_shift=torch.zeros(total - 1, dtype=torch.bfloat16), pse_type=1)
     assert st == _abi.FA_ERR_INNER_NULLPTR
+
+
+# ---------------------------------------------------------------------------
+# Global positions and the merge entry point (validation only on the CPU)
+# ---------------------------------------------------------------------------
+
+def test_plan_start_indices_shift_must_be_common():
+    lens = [300, 200]
+    cum = [300, 500]
+    q, k, v = qkv((500, 2, 128), torch.bfloat16)
+    base = dict(input_layout="TND", head_num=2, actual_seq_qlen=cum, actual_seq_kvlen=cum, next_tokens=0)
+    assert plan(q, k, v, q_start_idx=[64, 64], kv_start_idx=[0, 0], **base)[0] == 0
+    assert plan(q, k, v, q_start_idx=64, kv_start_idx=[0, 0], **base)[0] == 0
+    # different kvStart - qStart per sequence
+    assert plan(q, k, v, q_start_idx=[0, 0], kv_start_idx=[0, 5], **base)[0] == _abi.FA_ERR_INNER_NULLPTR
+    # one value per sequence or a single value only
+    assert plan(q, k, v, q_start_idx=[0, 0, 0], **base)[0] == _abi.FA_ERR_INNER_NULLPTR
+    assert plan(q, k, v, kv_start_idx=-1, **base)[0] == _abi.FA_ERR_INNER_NULLPTR
+
+
+def _merge_status(outs, maxes, sums, out, smax, ssum, layout="BNSD", heads=2):
+    lib = _abi.load()
+    n = len(outs)
+    P = ctypes.POINTER(_abi.FaTensor)
+    ft = lambda t: _abi.make_tensor(t.data_ptr(), 1 if t.dtype == torch.float16 else 0, t.shape, t.stride())  # noqa: E731
+    keep = [ft(t) for t in outs + maxes + sums]
+    arr = lambda ts: (P * max(1, len(ts)))(*[ctypes.pointer(t) for t in ts])  # noqa: E731
+    o, m, s_ = ft(out), ft(smax), ft(ssum)
+    return lib.fa_lse_merge(arr(keep[:n]), arr(keep[n:2 * n]), arr(keep[2 * n:]), n, None, heads, layout.encode(),
+                            b"", None, 0, ctypes.byref(o), ctypes.byref(m), ctypes.byref(s_), None)
+
+
+def test_merge_validation():
+    out = torch.zeros(1, 2, 40, 64, dtype=torch.float16)
+    st = torch.zeros(1, 2, 40, 8)
+    assert _merge_status([], [], [], out, st, st) == _abi.FA_ERR_INNER_NULLPTR  # no part
+    bad = torch.zeros(1, 2, 41, 64, dtype=torch.float16)
+    assert _merge_status([bad], [st], [st], out, st, st) == _abi.FA_ERR_INNER_NULLPTR  # shape
+    assert _merge_status([out], [torch.zeros(1, 2, 40, 4)], [st], out, st, st) == _abi.FA_ERR_INNER_NULLPTR

@@ -377,3 +377,61 @@ def test_full_size_band_with_compressed_bias_sampled():
     for t in res:
         assert not torch.isnan(t).any()
     compare_rows(w, res, sample_rows(w, 16, seed=55))
+
+
+# ---------------------------------------------------------------------------
+# Global positions and the merge of partial results (a forward split along the
+# keys: each key chunk run at its kvStartIdx, then fa_lse_merge with the sink)
+# ---------------------------------------------------------------------------
+
+from tests.parity import check_out, check_stats, oracle_full  # noqa: E402
+
+
+def _kv_chunks_merged(w, bounds):
+    q = w.q.cuda()
+    kw = dict(input_layout=w.layout, head_num=w.head_num, scale=w.scale, pre_tokens=w.pre_tokens,
+              next_tokens=w.next_tokens)
+    if w.pse is not None:
+        kw.update(real_shift=w.pse.cuda(), pse_type=w.pse_type)
+    parts = []
+    for a, b in bounds:
+        kc = w.k[:, :, a:b].contiguous().cuda()
+        vc = w.v[:, :, a:b].contiguous().cuda()
+        parts.append(fa.fa_fwd(q, kc, vc, kv_start_idx=a, **kw))
+    sink = None if w.sink is None else w.sink.cuda()
+    res = fa.lse_merge([p_[0] for p_ in parts], [p_[1] for p_ in parts], [p_[2] for p_ in parts],
+                       input_layout=w.layout, head_num=w.head_num, sink=sink)
+    torch.cuda.synchronize()
+    return res
+
+
+@pytest.mark.parametrize("dtype,d,kw", [
+    ("f16", 128, dict(pre_tokens=300, next_tokens=0)),
+    ("bf16", 64, dict(pre_tokens=120, next_tokens=40)),
+    ("f32", 64, dict(next_tokens=0)),
+])
+def test_key_chunks_at_their_start_merged(dtype, d, kw):
+    n, s = 2, 700
+    w = W("BNSD", dtype, (1, n, s, d), n, 3500, sink=normal((n,), "f32", 3504), **kw)
+    if dtype == "f16":
+        w.pse, w.pse_type = alibi_slopes(n), 2
+    out, smax, ssum = _kv_chunks_merged(w, [(0, 256), (256, 500), (500, 700)])
+    want = oracle_full(w)
+    check_out(f64(out), want["out"], dtype)
+    check_stats(f64(smax), want["softmax_max"], "softmaxMax")
+    check_stats(f64(ssum), want["softmax_sum"], "softmaxSum")
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+def test_query_chunk_at_its_start(dtype, d):
+    n, s, a, b = 2, 640, 200, 530
+    w = W("BNSD", dtype, (1, n, s, d), n, 3600, pre_tokens=150, next_tokens=0)
+    w.pse, w.pse_type = alibi_slopes(n), 2
+    out, smax, ssum = fa.fa_fwd(w.q[:, :, a:b].contiguous().cuda(), w.k.cuda(), w.v.cuda(), input_layout="BNSD",
+                                head_num=n, scale=w.scale, pre_tokens=150, next_tokens=0,
+                                real_shift=w.pse.cuda(), pse_type=2, q_start_idx=a)
+    torch.cuda.synchronize()
+    want = oracle_full(w)
+    check_out(f64(out), want["out"][:, :, a:b], dtype)
+    check_stats(f64(smax), want["softmax_max"][:, :, a:b], "softmaxMax")
+    check_stats(f64(ssum), want["softmax_sum"][:, :, a:b], "softmaxSum")

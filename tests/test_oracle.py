@@ -413,3 +413,55 @@ def test_tnd_flat_bias_equals_each_sequence_with_its_own_bias():
         np.testing.assert_allclose(res["out"][cq[b]:cq[b + 1]], one["out"][0].transpose(1, 0, 2), atol=1e-13)
         np.testing.assert_allclose(res["softmax_max"][:, cq[b]:cq[b + 1], 0], one["softmax_max"][0, :, :, 0],
                                    rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Global positions (qStartIdx / kvStartIdx) and the merge of partial results
+# ---------------------------------------------------------------------------
+
+def _chunked_forward(q, k, v, n, bounds, **kw):
+    sink = kw.pop("sink", None)
+    parts = [ref.forward(q, k[:, :, a:b], v[:, :, a:b], layout="BNSD", head_num=n, kv_start=a, **kw)
+             for a, b in bounds]
+    o, m, l = ref.merge([p_["out"] for p_ in parts], [p_["softmax_max"][..., 0] for p_ in parts],
+                        [p_["softmax_sum"][..., 0] for p_ in parts],
+                        sink=None if sink is None else np.asarray(sink)[None, :, None])
+    return o, m, l
+
+
+@pytest.mark.parametrize("kw", [dict(pre_tokens=90, next_tokens=0),
+                                dict(pre_tokens=40, next_tokens=25),
+                                dict(next_tokens=0, pse_type=2)])
+def test_key_chunks_at_their_start_merge_to_the_whole(kw):
+    # the whole forward regrouped by key chunk: each chunk sees its keys at
+    # global positions (kv_start) and the merge combines the chunks' rows
+    n, s, d = 2, 200, 16
+    q, k, v = rand((1, n, s, d), 931), rand((1, n, s, d), 932), rand((1, n, s, d), 933)
+    sink = np.array([0.7, -1.3])
+    kw = dict(kw)
+    if kw.get("pse_type") == 2:
+        kw["pse"] = np.array([0.25, 0.0625])
+    whole = ref.forward(q, k, v, layout="BNSD", head_num=n, scale=0.3, sink=sink, **kw)
+    o, m, l = _chunked_forward(q, k, v, n, [(0, 70), (70, 130), (130, 200)], scale=0.3, sink=sink, **kw)
+    np.testing.assert_allclose(o, whole["out"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(m, whole["softmax_max"][..., 0], rtol=1e-13)
+    np.testing.assert_allclose(l, whole["softmax_sum"][..., 0], rtol=1e-12)
+
+
+def test_query_chunk_at_its_start_equals_rows_of_the_whole():
+    n, s, d = 2, 160, 8
+    q, k, v = rand((1, n, s, d), 941), rand((1, n, s, d), 942), rand((1, n, s, d), 943)
+    kw = dict(layout="BNSD", head_num=n, scale=0.4, pre_tokens=50, next_tokens=3, pse=np.array([0.5, 0.125]),
+              pse_type=2)
+    whole = ref.forward(q, k, v, **kw)
+    part = ref.forward(q[:, :, 100:140], k, v, q_start=100, **kw)
+    np.testing.assert_allclose(part["out"], whole["out"][:, :, 100:140], atol=1e-13)
+    np.testing.assert_allclose(part["softmax_sum"], whole["softmax_sum"][:, :, 100:140], rtol=1e-13)
+
+
+def test_merge_of_empty_parts():
+    # rows with no key in any part: o = 0, m = -inf, l = 0; with a sink m = sink, l = 1
+    o, m, l = ref.merge([np.zeros((3, 4))] * 2, [np.full(3, -np.inf)] * 2, [np.zeros(3)] * 2)
+    assert (o == 0).all() and np.isneginf(m).all() and (l == 0).all()
+    o, m, l = ref.merge([np.zeros((3, 4))], [np.full(3, -np.inf)], [np.zeros(3)], sink=np.full(3, 2.0))
+    assert (o == 0).all() and (m == 2.0).all() and (l == 1.0).all()

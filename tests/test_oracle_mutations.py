@@ -45,6 +45,11 @@ MUTATIONS = [
      "out[k] = pse[bb, nn, min(i, 1023), :kv_len]"),
     ("flat bias sequence offset skips the heads", "off = sum(n_heads * s[1] * s[3] for s in seqs[:b])",
      "off = sum(s[1] * s[3] for s in seqs[:b])"),
+    ("global position shift with the wrong sign", "diff = j[None, :] - i[:, None] + delta",
+     "diff = j[None, :] - i[:, None] - delta"),
+    ("ALiBi ignores the global positions", "j = np.arange(kv_len, dtype=np.float64) + delta",
+     "j = np.arange(kv_len, dtype=np.float64)"),
+    ("merge weights without the partial sums", "w = np.where(l_k > 0, l_k * np.exp(", "w = np.where(l_k > 0, 1.0 * np.exp("),
 ]
 
 
@@ -81,6 +86,11 @@ def _run_pins():
         pins.test_compressed_alibi_bias_equals_slopes(nxt)
     pins.test_compressed_bias_rows_are_read_along_the_diagonal()
     pins.test_tnd_flat_bias_equals_each_sequence_with_its_own_bias()
+    for kw in (dict(pre_tokens=90, next_tokens=0), dict(pre_tokens=40, next_tokens=25),
+               dict(next_tokens=0, pse_type=2)):
+        pins.test_key_chunks_at_their_start_merge_to_the_whole(kw)
+    pins.test_query_chunk_at_its_start_equals_rows_of_the_whole()
+    pins.test_merge_of_empty_parts()
 
 
 def _with_ref(mod):
