@@ -14,11 +14,13 @@ INT64_MAX = 2**63 - 1
 
 
 def head_forward(q, k, v, scale, pse=None, excluded=None,
-                 pre_tokens=INT64_MAX, next_tokens=INT64_MAX, sink=None):
+                 pre_tokens=INT64_MAX, next_tokens=INT64_MAX, sink=None, q_rope=None, k_rope=None):
     """q: Sq lists of D floats; k: Skv lists of D; v: Skv lists of Dv.
 
     pse: Sq lists of Skv floats or None; excluded: Sq lists of Skv bools or
-    None.  Returns (o, m, l) as nested Python lists / floats.
+    None; q_rope / k_rope: Sq / Skv lists of Dr floats or None (the page's
+    forward formula scales queryRope keyRope^T together with query key^T).
+    Returns (o, m, l) as nested Python lists / floats.
     """
     sq, skv, dv = len(q), len(k), (len(v[0]) if v else 0)
     outs, maxes, sums = [], [], []
@@ -29,7 +31,10 @@ def head_forward(q, k, v, scale, pse=None, excluded=None,
                 continue
             if excluded is not None and excluded[i][j]:
                 continue
-            dot = math.fsum(q[i][d] * k[j][d] for d in range(len(q[i])))
+            terms = [q[i][d] * k[j][d] for d in range(len(q[i]))]
+            if q_rope is not None:
+                terms += [q_rope[i][e] * k_rope[j][e] for e in range(len(q_rope[i]))]
+            dot = math.fsum(terms)
             s = scale * dot + (pse[i][j] if pse is not None else 0.0)
             scores.append((s, j))
         candidates = [s for s, _ in scores] + ([sink] if sink is not None else [])

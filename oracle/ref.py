@@ -10,7 +10,8 @@ pages describe and that the tiled kernel reaches up to rounding order
 sink formula; aclnnFlashAttentionScore, parameter list for attenMask,
 scaleValue, preTockens/nextTockens, softmaxMax/softmaxSum):
 
-    s_ij    = scale * sum_d q_id k_jd + pse_ij          (pse_ij = 0 without pse)
+    s_ij    = scale * (sum_d q_id k_jd + sum_e qr_ie kr_je) + pse_ij
+              (pse_ij = 0 without pse; the rope term only with queryRope/keyRope)
     keep_ij = (-preTokens <= j - i <= nextTokens) and not attenMask_ij
     m_i     = max({s_ij : keep_ij} U {sink_n if a sink is given})
     l_i     = sum_{keep} exp(s_ij - m_i) + [sink] exp(sink_n - m_i)
@@ -28,7 +29,10 @@ Readings where the pages are silent (each listed in the design doc):
     sink it gives o = 0, m = sink, l = 1;
   * softmaxMax / softmaxSum are m_i (natural-log units) and l_i, written to
     all 8 lanes of the trailing axis;
-  * ALiBi slopes (pse type 2) give pse_ij = -slope_n * |i - j|.
+  * ALiBi slopes (pse type 2) give pse_ij = -slope_n * |i - j|;
+  * queryRope / keyRope (aclnnFlashAttentionVarLenScoreV5 formula,
+    scale*(query key^T + queryRope keyRope^T)) add a second dot product over
+    their own head dim inside the scaling.
 
 Inputs are taken exactly as the kernel sees them: arrays already rounded to
 their storage dtype, then widened to float64 here.
@@ -84,14 +88,16 @@ def from_heads(o, layout):
 # ---------------------------------------------------------------------------
 
 def head_forward(q, k, v, scale, rows=None, pse=None, excluded=None,
-                 pre_tokens=INT64_MAX, next_tokens=INT64_MAX, sink=None, delta=0):
+                 pre_tokens=INT64_MAX, next_tokens=INT64_MAX, sink=None, delta=0,
+                 q_rope=None, k_rope=None):
     """Attention of one (batch, head).
 
     q: [R, D] query rows whose in-sequence indices are `rows` (default 0..R-1);
     k: [Skv, D]; v: [Skv, Dv]; pse: [R, Skv] additive bias or None;
     excluded: bool [R, Skv] (True = does not take part) or None;
     sink: float or None; delta: kvStartIdx - qStartIdx, the band compares the
-    global positions (kvStart + j) - (qStart + i) = j - i + delta.
+    global positions (kvStart + j) - (qStart + i) = j - i + delta;
+    q_rope [R, Dr], k_rope [Skv, Dr]: the rope parts of query and key, or None.
     Returns o [R, Dv], m [R], l [R] in float64.
     """
     q = np.asarray(q, dtype=np.float64)
@@ -108,7 +114,10 @@ def head_forward(q, k, v, scale, rows=None, pse=None, excluded=None,
     for r0 in range(0, n_rows, ROW_BLOCK):
         r1 = min(n_rows, r0 + ROW_BLOCK)
         i = rows[r0:r1]
-        s = scale * (q[r0:r1] @ k.T)
+        qk = q[r0:r1] @ k.T
+        if q_rope is not None:
+            qk = qk + np.asarray(q_rope[r0:r1], dtype=np.float64) @ np.asarray(k_rope, dtype=np.float64).T
+        s = scale * qk
         if pse is not None:
             s = s + np.asarray(pse[r0:r1], dtype=np.float64)
         diff = j[None, :] - i[:, None] + delta
@@ -153,6 +162,25 @@ def _head_inputs(layout, qh, kh, vh, b, n, n_kv, seq):
     if layout == "TND":
         return qh[q0:q0 + ql, n, :], kh[k0:k0 + kl, n_kv, :], vh[k0:k0 + kl, n_kv, :]
     return qh[b, n, :ql, :], kh[b, n_kv, :kl, :], vh[b, n_kv, :kl, :]
+
+
+def _rope_views(query_rope, key_rope, layout, head_num):
+    """Logical views of queryRope / keyRope (the query's / key's layout, own head dim), or Nones."""
+    if query_rope is None and key_rope is None:
+        return None, None
+    if query_rope is None or key_rope is None:
+        raise ValueError("queryRope and keyRope go together")
+    dr = _head_dim(query_rope, layout, head_num)
+    return heads_view(query_rope, layout, dr), heads_view(key_rope, layout, dr)
+
+
+def _rope_inputs(layout, qrh, krh, b, n, n_kv, seq):
+    if qrh is None:
+        return None, None
+    q0, ql, k0, kl = seq
+    if layout == "TND":
+        return qrh[q0:q0 + ql, n, :], krh[k0:k0 + kl, n_kv, :]
+    return qrh[b, n, :ql, :], krh[b, n_kv, :kl, :]
 
 
 def _pse_rows(pse, pse_type, b, n, rows, kv_len, seqs=None, n_heads=None, delta=0):
@@ -225,7 +253,8 @@ def _deltas(q_start, kv_start, n_seqs):
 
 def forward(query, key, value, *, layout, head_num, scale, pse=None, pse_type=None,
             atten_mask=None, pre_tokens=INT64_MAX, next_tokens=INT64_MAX, sink=None,
-            actual_seq_q=None, actual_seq_kv=None, softmax_out_layout="", q_start=None, kv_start=None):
+            actual_seq_q=None, actual_seq_kv=None, softmax_out_layout="", q_start=None, kv_start=None,
+            query_rope=None, key_rope=None):
     """Full forward.  Returns dict(out, softmax_max, softmax_sum) in float64.
 
     out has the query layout (value head dim); the statistics are
@@ -236,6 +265,7 @@ def forward(query, key, value, *, layout, head_num, scale, pse=None, pse_type=No
     qh = heads_view(query, layout, head_dim)
     kh = heads_view(key, layout, head_dim)
     vh = heads_view(value, layout, _value_head_dim(value, key, layout, head_dim))
+    qrh, krh = _rope_views(query_rope, key_rope, layout, head_num)
     n_q = head_num
     n_kv = kh.shape[1]
     group = n_q // n_kv
@@ -260,8 +290,9 @@ def forward(query, key, value, *, layout, head_num, scale, pse=None, pse_type=No
         rows = np.arange(q_len)
         for n in range(n_q):
             qs, ks, vs = _head_inputs(layout, qh, kh, vh, b, n, n // group, seq)
+            qr, kr = _rope_inputs(layout, qrh, krh, b, n, n // group, seq)
             o, m, l = head_forward(
-                qs, ks, vs, scale, rows=rows,
+                qs, ks, vs, scale, rows=rows, q_rope=qr, k_rope=kr,
                 pse=_pse_rows(pse, pse_type, b, n, rows, kv_len, seqs, n_q, deltas[b]),
                 excluded=_mask_rows(atten_mask, b, n, rows, kv_len),
                 pre_tokens=pre_tokens, next_tokens=next_tokens,
@@ -285,7 +316,8 @@ def forward(query, key, value, *, layout, head_num, scale, pse=None, pse_type=No
 
 def forward_rows(query, key, value, rows, *, layout, head_num, scale, pse=None, pse_type=None,
                  atten_mask=None, pre_tokens=INT64_MAX, next_tokens=INT64_MAX, sink=None,
-                 actual_seq_q=None, actual_seq_kv=None, q_start=None, kv_start=None):
+                 actual_seq_q=None, actual_seq_kv=None, q_start=None, kv_start=None,
+                 query_rope=None, key_rope=None):
     """Selected output rows only: `rows` is a list of (b, n, i), i the in-sequence index.
 
     Returns o [R, Dv], m [R], l [R]; used to check full-size runs row by row.
@@ -294,6 +326,7 @@ def forward_rows(query, key, value, rows, *, layout, head_num, scale, pse=None, 
     qh = heads_view(query, layout, head_dim)
     kh = heads_view(key, layout, head_dim)
     vh = heads_view(value, layout, _value_head_dim(value, key, layout, head_dim))
+    qrh, krh = _rope_views(query_rope, key_rope, layout, head_num)
     group = head_num // kh.shape[1]
     seqs = _sequences(layout, qh, kh, actual_seq_q, actual_seq_kv)
     deltas = _deltas(q_start, kv_start, len(seqs))
@@ -302,9 +335,11 @@ def forward_rows(query, key, value, rows, *, layout, head_num, scale, pse=None, 
     for (b, n, i) in rows:
         seq = seqs[b]
         qs, ks, vs = _head_inputs(layout, qh, kh, vh, b, n, n // group, seq)
+        qr, kr = _rope_inputs(layout, qrh, krh, b, n, n // group, seq)
         r = np.array([i])
         o, m, l = head_forward(
             qs[i:i + 1], ks, vs, scale, rows=r,
+            q_rope=None if qr is None else qr[i:i + 1], k_rope=kr,
             pse=_pse_rows(pse, pse_type, b, n, r, seq[3], seqs, head_num, deltas[b]),
             excluded=_mask_rows(atten_mask, b, n, r, seq[3]),
             pre_tokens=pre_tokens, next_tokens=next_tokens,

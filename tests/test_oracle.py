@@ -54,6 +54,28 @@ def test_worked_example_sink_closed_form():
     assert torch.tensor(res["out"]).to(torch.bfloat16).float().eq(1.0).all()
 
 
+def test_worked_example_with_rope_closed_form():
+    """The page's exact call, queryRope/keyRope [256, 1, 64] of ones included:
+    every score is scale * (128 + 64)."""
+    g = json.load(open(os.path.join(GOLDEN, "sink_example_tnd.json")))
+    t, n, d, dr = g["T"], g["N"], g["D"], g["rope_dim"]
+    one = f64(torch.ones(t, n, d, dtype=torch.bfloat16))
+    rope = f64(torch.ones(t, n, dr, dtype=torch.bfloat16))
+    res = ref.forward(one, one, one, layout="TND", head_num=n, scale=g["scale"],
+                      atten_mask=np.zeros((t, t), np.uint8),
+                      pre_tokens=g["pre_tokens"], next_tokens=g["next_tokens"],
+                      sink=np.array([g["host_fill"]["sink"]]),
+                      actual_seq_q=g["actual_seq_q"], actual_seq_kv=g["actual_seq_kv"],
+                      softmax_out_layout=g["softmax_out_layout"], query_rope=rope, key_rope=rope)
+    exp = g["expected_with_rope"]
+    np.testing.assert_allclose(res["softmax_max"], exp["softmax_max"], rtol=1e-12)
+    np.testing.assert_allclose(res["softmax_sum"], exp["softmax_sum"], rtol=1e-12)
+    np.testing.assert_allclose(res["out"], exp["out"], rtol=1e-12)
+    s = g["scale"] * (d + dr)
+    assert abs(exp["softmax_max"] - s) < 1e-9
+    assert abs(exp["softmax_sum"] - (t + math.exp(3.0 - s))) < 1e-9
+
+
 # ---------------------------------------------------------------------------
 # Reduction to a library routine: torch scaled_dot_product_attention (float64).
 # ---------------------------------------------------------------------------
@@ -136,6 +158,20 @@ def test_ref_matches_brute(with_sink, with_pse, with_mask, pre, nxt):
     np.testing.assert_array_equal(np.isinf(m), np.isinf(np.array(mb)))
     fin = np.isfinite(m)
     np.testing.assert_allclose(m[fin], np.array(mb)[fin], rtol=1e-13)
+    np.testing.assert_allclose(l, np.array(lb), rtol=1e-12)
+
+
+@pytest.mark.parametrize("with_sink,pre,nxt", [(False, INT64_MAX, INT64_MAX), (True, 2, 0)])
+def test_rope_matches_brute(with_sink, pre, nxt):
+    sq, skv, d, dr, dv = 5, 6, 3, 2, 2
+    q, k, v = rand((sq, d), 31), rand((skv, d), 32), rand((skv, dv), 33)
+    qr, kr = rand((sq, dr), 34), rand((skv, dr), 35)
+    sink = -0.3 if with_sink else None
+    o, m, l = ref.head_forward(q, k, v, 0.7, pre_tokens=pre, next_tokens=nxt, sink=sink, q_rope=qr, k_rope=kr)
+    ob, mb, lb = brute.head_forward(q.tolist(), k.tolist(), v.tolist(), 0.7, pre_tokens=pre, next_tokens=nxt,
+                                    sink=sink, q_rope=qr.tolist(), k_rope=kr.tolist())
+    np.testing.assert_allclose(o, np.array(ob), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(m, np.array(mb), rtol=1e-13)
     np.testing.assert_allclose(l, np.array(lb), rtol=1e-12)
 
 
@@ -465,3 +501,36 @@ def test_merge_of_empty_parts():
     assert (o == 0).all() and np.isneginf(m).all() and (l == 0).all()
     o, m, l = ref.merge([np.zeros((3, 4))], [np.full(3, -np.inf)], [np.zeros(3)], sink=np.full(3, 2.0))
     assert (o == 0).all() and (m == 2.0).all() and (l == 1.0).all()
+
+
+# ---------------------------------------------------------------------------
+# queryRope / keyRope (aclnnFlashAttentionVarLenScoreV5 formula): the sum of
+# the two dot products is one dot product over the joined head dims.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("layout", ["BSH", "TND"])
+def test_rope_equals_joined_head_dim(layout):
+    n_q, n_kv, d, dr, dv = 4, 2, 8, 4, 6
+    kw = dict(pre_tokens=9, next_tokens=0, sink=np.array([0.2, -1.0, 0.5, 1.5]))
+    if layout == "TND":
+        lens_q, lens_kv = [7, 0, 12], [9, 3, 12]
+        tq, tkv = sum(lens_q), sum(lens_kv)
+        q, qr = rand((tq, n_q, d), 41), rand((tq, n_q, dr), 42)
+        k, kr = rand((tkv, n_kv, d), 43), rand((tkv, n_kv, dr), 44)
+        v = rand((tkv, n_kv, dv), 45)
+        kw.update(actual_seq_q=cumulative(lens_q, False), actual_seq_kv=cumulative(lens_kv, False))
+        qj, kj = np.concatenate([q, qr], axis=-1), np.concatenate([k, kr], axis=-1)
+    else:
+        bsz, sq, skv = 2, 11, 13
+        q, qr = rand((bsz, sq, n_q * d), 41), rand((bsz, sq, n_q * dr), 42)
+        k, kr = rand((bsz, skv, n_kv * d), 43), rand((bsz, skv, n_kv * dr), 44)
+        v = rand((bsz, skv, n_kv * dv), 45)
+
+        def join(a, b, n):  # per head: the head's D columns, then its Dr columns
+            return np.concatenate([a.reshape(bsz, -1, n, d), b.reshape(bsz, -1, n, dr)],
+                                  axis=-1).reshape(bsz, -1, n * (d + dr))
+        qj, kj = join(q, qr, n_q), join(k, kr, n_kv)
+    with_rope = ref.forward(q, k, v, layout=layout, head_num=n_q, scale=0.3, query_rope=qr, key_rope=kr, **kw)
+    joined = ref.forward(qj, kj, v, layout=layout, head_num=n_q, scale=0.3, **kw)
+    for key in ("out", "softmax_max", "softmax_sum"):
+        np.testing.assert_allclose(with_rope[key], joined[key], rtol=1e-12, atol=1e-14)

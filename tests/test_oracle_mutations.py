@@ -16,7 +16,15 @@ MUTATIONS = [
     ("band left bound exclusive", "(diff >= -pre_tokens)", "(diff > -pre_tokens)"),
     ("band right bound exclusive", "(diff <= next_tokens)", "(diff < next_tokens)"),
     ("band direction swapped", "diff = j[None, :] - i[:, None]", "diff = i[:, None] - j[None, :]"),
-    ("scale dropped", "s = scale * (q[r0:r1] @ k.T)", "s = (q[r0:r1] @ k.T)"),
+    ("scale dropped", "s = scale * qk", "s = qk"),
+    ("rope term dropped", "qk = qk + np.asarray(q_rope[r0:r1], dtype=np.float64) @ np.asarray(k_rope, dtype=np.float64).T",
+     "qk = qk"),
+    ("rope term outside the scale",
+     "qk = qk + np.asarray(q_rope[r0:r1], dtype=np.float64) @ np.asarray(k_rope, dtype=np.float64).T",
+     "qk = qk + np.asarray(q_rope[r0:r1], dtype=np.float64) @ np.asarray(k_rope, dtype=np.float64).T / scale"),
+    ("rope key rows from the query", "np.asarray(k_rope, dtype=np.float64).T", "np.asarray(q_rope, dtype=np.float64).T"),
+    ("rope key head map by query head", "return qrh[b, n, :ql, :], krh[b, n_kv, :kl, :]",
+     "return qrh[b, n, :ql, :], krh[b, n % krh.shape[1], :kl, :]"),
     ("scale applied to pse too", "s = s + np.asarray(pse[r0:r1], dtype=np.float64)",
      "s = s + scale * np.asarray(pse[r0:r1], dtype=np.float64)"),
     ("pse sign flipped", "s = s + np.asarray(pse[r0:r1], dtype=np.float64)",
@@ -63,6 +71,11 @@ def _mutant(src, old, new, tag):
 def _run_pins():
     """Every pin of test_oracle.py, with fixed arguments; raises on the first failure."""
     pins.test_worked_example_sink_closed_form()
+    pins.test_worked_example_with_rope_closed_form()
+    for args in [(False, INT64_MAX, INT64_MAX), (True, 2, 0)]:
+        pins.test_rope_matches_brute(*args)
+    for layout in ("BSH", "TND"):
+        pins.test_rope_equals_joined_head_dim(layout)
     for args in [(37, 53, 16, 16, INT64_MAX, INT64_MAX), (64, 64, 32, 24, 10, 0), (50, 70, 8, 8, 5, 30)]:
         pins.test_head_matches_sdpa(*args)
     pins.test_sink_matches_sdpa_with_extra_key()
