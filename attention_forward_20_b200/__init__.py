@@ -85,9 +85,10 @@ def _out_shapes(query, layout, head_num, dv, softmax_out_layout):
 def _stage1(query, key, value, out, smax, ssum, *, input_layout, head_num, scale, real_shift,
             pse_type, atten_mask, mask_mode, sink, actual_seq_qlen, actual_seq_kvlen,
             pre_tokens, next_tokens, keep_prob, inner_precise, softmax_out_layout,
-            q_start_idx=None, kv_start_idx=None):
+            q_start_idx=None, kv_start_idx=None, query_rope=None, key_rope=None):
     lib = _abi.load()
     tq, tk, tv = _ft(query), _ft(key), _ft(value)
+    tqr, tkr = _ft(query_rope), _ft(key_rope)
     tpse, tmask, tsink = _ft(real_shift), _ft(atten_mask), _ft(sink)
     to, tmax, tsum = _ft(out), _ft(smax), _ft(ssum)
     aq, nq = _i64_array(actual_seq_qlen)
@@ -97,7 +98,7 @@ def _stage1(query, key, value, out, smax, ssum, *, input_layout, head_num, scale
     ws = ctypes.c_uint64(0)
     ex = ctypes.c_void_p(None)
     status = lib.fa_fwd_get_workspace_size_v5(
-        _ptr(tq), _ptr(tk), _ptr(tv), _ptr(tpse), _ptr(tmask), _ptr(tsink),
+        _ptr(tq), _ptr(tqr), _ptr(tk), _ptr(tkr), _ptr(tv), _ptr(tpse), _ptr(tmask), _ptr(tsink),
         aq, nq, akv, nkv, qst, nqst, kvst, nkvst,
         float(scale), float(keep_prob), int(pre_tokens), int(next_tokens),
         int(head_num), input_layout.encode(), int(inner_precise),
@@ -128,14 +129,17 @@ def fa_fwd(query, key, value, *, input_layout, head_num, scale=None, real_shift=
            atten_mask=None, mask_mode=FA_MASK_TENSOR, sink=None, actual_seq_qlen=None,
            actual_seq_kvlen=None, pre_tokens=INT64_MAX, next_tokens=INT64_MAX, keep_prob=1.0,
            inner_precise=0, softmax_out_layout="", out=None, softmax_max=None, softmax_sum=None,
-           q_start_idx=None, kv_start_idx=None):
+           q_start_idx=None, kv_start_idx=None, query_rope=None, key_rope=None):
     """The operator: returns (attention_out, softmax_max, softmax_sum).
 
     Arguments mirror fa_fwd_get_workspace_size_v5 (include/fa_fwd.h).  Tensors
     must be CUDA tensors on one device; actual_seq_* are host sequences of
     cumulative lengths without a leading zero; q_start_idx / kv_start_idx are
-    None, one int or one int per sequence.  The work is enqueued on the
-    current stream of the query's device.
+    None, one int or one int per sequence; query_rope / key_rope (bf16, the
+    query's / key's layout with their own head dim) add
+    scale * query_rope key_rope^T to the scores.  The default scale is
+    D ** -0.5 with D the query's head dim, rope or not.  The work is
+    enqueued on the current stream of the query's device.
     """
     if not query.is_cuda:
         raise ValueError("fa_fwd runs on CUDA tensors only (no CPU path)")
@@ -154,7 +158,7 @@ def fa_fwd(query, key, value, *, input_layout, head_num, scale=None, real_shift=
         atten_mask=atten_mask, mask_mode=mask_mode, sink=sink, actual_seq_qlen=actual_seq_qlen,
         actual_seq_kvlen=actual_seq_kvlen, pre_tokens=pre_tokens, next_tokens=next_tokens,
         keep_prob=keep_prob, inner_precise=inner_precise, softmax_out_layout=softmax_out_layout,
-        q_start_idx=q_start_idx, kv_start_idx=kv_start_idx)
+        q_start_idx=q_start_idx, kv_start_idx=kv_start_idx, query_rope=query_rope, key_rope=key_rope)
     if status != FA_SUCCESS:
         raise FaError(status, "fa_fwd_get_workspace_size_v5")
     ws = torch.empty(max(1, ws_bytes), dtype=torch.uint8, device=dev) if ws_bytes else None
@@ -170,7 +174,7 @@ def plan(query, key, value, *, input_layout, head_num, scale=None, real_shift=No
          atten_mask=None, mask_mode=FA_MASK_TENSOR, sink=None, actual_seq_qlen=None,
          actual_seq_kvlen=None, pre_tokens=INT64_MAX, next_tokens=INT64_MAX, keep_prob=1.0,
          inner_precise=0, softmax_out_layout="", out=None, softmax_max=None, softmax_sum=None,
-         q_start_idx=None, kv_start_idx=None):
+         q_start_idx=None, kv_start_idx=None, query_rope=None, key_rope=None):
     """Stage 1 only (no device work): returns (status, workspace_bytes, plan_text)."""
     _, dv, scale, pse_type = _defaults(query, key, value, input_layout, head_num, scale, real_shift, pse_type)
     out_shape, stats_shape = _out_shapes(query, input_layout, head_num, dv, softmax_out_layout)
@@ -187,7 +191,7 @@ def plan(query, key, value, *, input_layout, head_num, scale=None, real_shift=No
         atten_mask=atten_mask, mask_mode=mask_mode, sink=sink, actual_seq_qlen=actual_seq_qlen,
         actual_seq_kvlen=actual_seq_kvlen, pre_tokens=pre_tokens, next_tokens=next_tokens,
         keep_prob=keep_prob, inner_precise=inner_precise, softmax_out_layout=softmax_out_layout,
-        q_start_idx=q_start_idx, kv_start_idx=kv_start_idx)
+        q_start_idx=q_start_idx, kv_start_idx=kv_start_idx, query_rope=query_rope, key_rope=key_rope)
     text = ""
     if status == FA_SUCCESS:
         lib = _abi.load()

@@ -68,7 +68,8 @@ def load():
     ]
     lib.fa_fwd_get_workspace_size_v5.restype = ctypes.c_int32
     lib.fa_fwd_get_workspace_size_v5.argtypes = [
-        P(FaTensor), P(FaTensor), P(FaTensor),                  # query, key, value
+        P(FaTensor), P(FaTensor), P(FaTensor), P(FaTensor),     # query, queryRope, key, keyRope
+        P(FaTensor),                                            # value
         P(FaTensor), P(FaTensor), P(FaTensor),                  # realShift, attenMask, sink
         P(ctypes.c_int64), ctypes.c_int64,                      # actualSeqQLen, nSeqQ
         P(ctypes.c_int64), ctypes.c_int64,                      # actualSeqKvLen, nSeqKv

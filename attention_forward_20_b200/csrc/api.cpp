@@ -123,7 +123,8 @@ int64_t kv_blocks_for_tile(int64_t r0, int64_t q_len, int64_t kv_len, int64_t pr
 }  // namespace
 
 extern "C" fa_status fa_fwd_get_workspace_size_v5(
-    const fa_tensor* query, const fa_tensor* key, const fa_tensor* value,
+    const fa_tensor* query, const fa_tensor* queryRope, const fa_tensor* key, const fa_tensor* keyRope,
+    const fa_tensor* value,
     const fa_tensor* realShift, const fa_tensor* attenMask, const fa_tensor* sink,
     const int64_t* actualSeqQLen, int64_t nSeqQ,
     const int64_t* actualSeqKvLen, int64_t nSeqKv,
@@ -144,6 +145,8 @@ extern "C" fa_status fa_fwd_get_workspace_size_v5(
         return FA_ERR_PARAM_NULLPTR;
     if ((realShift && !realShift->data) || (attenMask && !attenMask->data) || (sink && !sink->data))
         return FA_ERR_PARAM_NULLPTR;
+    if ((queryRope && !queryRope->data) || (keyRope && !keyRope->data)) return FA_ERR_PARAM_NULLPTR;
+    const bool rope = queryRope != nullptr;
 
     // ---- 161002: dtypes and format strings ------------------------------
     Layout L;
@@ -157,6 +160,11 @@ extern "C" fa_status fa_fwd_get_workspace_size_v5(
     if (softmaxMax->dtype != FA_F32 || softmaxSum->dtype != FA_F32) return FA_ERR_PARAM_INVALID;
     if (attenMask && attenMask->dtype != FA_U8 && attenMask->dtype != FA_BOOL) return FA_ERR_PARAM_INVALID;
     if (sink && sink->dtype != FA_F32) return FA_ERR_PARAM_INVALID;
+    // queryRope / keyRope: BFLOAT16 only, the dtype of query/key/value
+    // (aclnnFlashAttentionVarLenScoreV5, parameter list)
+    if ((queryRope && (queryRope->dtype != FA_BF16 || dt != FA_BF16)) ||
+        (keyRope && (keyRope->dtype != FA_BF16 || dt != FA_BF16)))
+        return FA_ERR_PARAM_INVALID;
     if (realShift) {
         if (pseType == FA_PSE_DENSE && realShift->dtype != dt) return FA_ERR_PARAM_INVALID;
         if (pseType == FA_PSE_ALIBI && realShift->dtype != FA_F32) return FA_ERR_PARAM_INVALID;
@@ -189,6 +197,18 @@ extern "C" fa_status fa_fwd_get_workspace_size_v5(
     if (ov.N != qv.N || ov.S != qv.S || ov.D != vv.D || (L != L_TND && ov.B != qv.B))
         return FA_ERR_INNER_NULLPTR;
     if (qv.S > kMaxS || kv.S > kMaxS) return FA_ERR_INNER_NULLPTR;
+    // rope: both or neither; no realShift with it (same page: realShiftOptional
+    // is incompatible with queryRope/keyRope); the query's / key's layout,
+    // sizes and head counts with a head dim Dr of their own; D + Dr <= 256.
+    View qrv, krv;
+    if (rope || keyRope) {
+        if (!queryRope || !keyRope || realShift) return FA_ERR_INNER_NULLPTR;
+        if ((s = make_view(queryRope, L, headNum, 0, &qrv)) != FA_SUCCESS) return s;
+        if ((s = make_view(keyRope, L, kv.N, 0, &krv)) != FA_SUCCESS) return s;
+        if (qrv.N != qv.N || qrv.S != qv.S || qrv.B != qv.B || krv.N != kv.N || krv.S != kv.S || krv.B != kv.B ||
+            krv.D != qrv.D || qv.D + qrv.D > kMaxD)
+            return FA_ERR_INNER_NULLPTR;
+    }
 
     auto* ex = new (std::nothrow) fa_executor();
     if (!ex) return FA_ERR_INNER_NULLPTR;
@@ -340,6 +360,12 @@ extern "C" fa_status fa_fwd_get_workspace_size_v5(
     p.k_b = kv.sb; p.k_n = kv.sn; p.k_s = kv.ss;
     p.v_b = vv.sb; p.v_n = vv.sn; p.v_s = vv.ss;
     p.o_b = ov.sb; p.o_n = ov.sn; p.o_s = ov.ss;
+    if (rope) {
+        p.qr = queryRope->data; p.kr = keyRope->data;
+        p.qr_b = qrv.sb; p.qr_n = qrv.sn; p.qr_s = qrv.ss;
+        p.kr_b = krv.sb; p.kr_n = krv.sn; p.kr_s = krv.ss;
+        p.Dr = (int32_t)qrv.D;
+    }
     if (L != L_TND) {
         p.st_b = softmaxMax->strides[0]; p.st_n = softmaxMax->strides[1]; p.st_s = softmaxMax->strides[2];
     } else if (stats_same_as_input) {
@@ -390,6 +416,11 @@ extern "C" fa_status fa_fwd_get_workspace_size_v5(
     tma_ok = tma_ok && tma_dim_ok(p.q_s, qv.S) && tma_dim_ok(p.q_n, qv.N) && tma_dim_ok(p.q_b, qB);
     tma_ok = tma_ok && tma_dim_ok(p.k_s, kv.S) && tma_dim_ok(p.k_n, kv.N) && tma_dim_ok(p.k_b, qB);
     tma_ok = tma_ok && tma_dim_ok(p.v_s, vv.S) && tma_dim_ok(p.v_n, vv.N) && tma_dim_ok(p.v_b, qB);
+    // rope on the tcgen05 path: one 64-column chunk more in Q and K
+    if (rope)
+        tma_ok = tma_ok && p.Dr == 64 && aligned16(p.qr) && aligned16(p.kr) && tma_dim_ok(p.qr_s, qv.S) &&
+                 tma_dim_ok(p.qr_n, qv.N) && tma_dim_ok(p.qr_b, qB) && tma_dim_ok(p.kr_s, kv.S) &&
+                 tma_dim_ok(p.kr_n, kv.N) && tma_dim_ok(p.kr_b, qB);
     const bool sm100 = (dt == FA_F16 || dt == FA_BF16) && qv.D == vv.D && (qv.D == 64 || qv.D == 128) && tma_ok;
     ex->kind = sm100 ? fa::KERNEL_SM100 : fa::KERNEL_SIMT;
 
@@ -462,10 +493,10 @@ extern "C" fa_status fa_fwd_get_workspace_size_v5(
 
     char buf[256];
     std::snprintf(buf, sizeof(buf),
-                  "kernel=%s dtype=%s D=%d Dv=%d B=%d Nq=%d Nkv=%d Sq=%d Skv=%d varlen=%d items=%d grid=%d "
+                  "kernel=%s dtype=%s D=%d Dv=%d Dr=%d B=%d Nq=%d Nkv=%d Sq=%d Skv=%d varlen=%d items=%d grid=%d "
                   "dynamic=%d split_items=%d pieces=%d ws=%llu",
                   sm100 ? "sm100_tcgen05" : "simt_fp32acc", dt == FA_F32 ? "f32" : dt == FA_F16 ? "f16" : "bf16",
-                  p.D, p.Dv, p.B, p.Nq, p.Nkv, p.Sq, p.Skv, p.varlen, p.n_items, p.grid,
+                  p.D, p.Dv, p.Dr, p.B, p.Nq, p.Nkv, p.Sq, p.Skv, p.varlen, p.n_items, p.grid,
                   p.dynamic, p.n_items - p.n_whole, p.n_pieces, (unsigned long long)off);
     ex->desc = buf;
     (void)innerPrecise;
@@ -483,7 +514,7 @@ extern "C" fa_status fa_fwd_get_workspace_size(
     int64_t maskMode, int64_t pseType, const char* softmaxOutLayout,
     const fa_tensor* softmaxMax, const fa_tensor* softmaxSum, const fa_tensor* attentionOut,
     uint64_t* workspaceSize, fa_executor** executor) {
-    return fa_fwd_get_workspace_size_v5(query, key, value, realShift, attenMask, sink, actualSeqQLen, nSeqQ,
+    return fa_fwd_get_workspace_size_v5(query, nullptr, key, nullptr, value, realShift, attenMask, sink, actualSeqQLen, nSeqQ,
                                         actualSeqKvLen, nSeqKv, nullptr, 0, nullptr, 0, scaleValue, keepProb,
                                         preTokens, nextTokens, headNum, inputLayout, innerPrecise, maskMode, pseType,
                                         softmaxOutLayout, softmaxMax, softmaxSum, attentionOut, workspaceSize,
@@ -520,9 +551,9 @@ extern "C" fa_status fa_fwd(void* workspace, uint64_t workspaceSize, fa_executor
         p.sched_counter = reinterpret_cast<int*>(ws);
         p.part = ex->off_part ? reinterpret_cast<float*>(ws + ex->off_part) : nullptr;
         if (p.grid > 0 && p.dynamic && cudaMemsetAsync(ws, 0, sizeof(int), st) != cudaSuccess) return done(FA_ERR_CUDA);
-        fa::TmaDesc tq, tk, tv;
-        if (fa::make_sm100_tmaps(p, &tq, &tk, &tv) != cudaSuccess) return done(FA_ERR_CUDA);
-        err = fa::launch_sm100(p, tq, tk, tv, p.grid, st);
+        fa::TmaSet maps;
+        if (fa::make_sm100_tmaps(p, &maps) != cudaSuccess) return done(FA_ERR_CUDA);
+        err = fa::launch_sm100(p, maps, p.grid, st);
     } else {
         err = fa::launch_simt(p, st);
     }

@@ -20,11 +20,15 @@ struct FaParams {
     const void* pse;      // dense bias (query dtype) or fp32 ALiBi slopes
     const uint8_t* mask;  // nonzero = excluded; read only when mask_on
     const float* sink;    // fp32 [Nq] or nullptr
+    const void* qr;       // queryRope (query layout, head dim Dr) or nullptr
+    const void* kr;       // keyRope (key layout, head dim Dr) or nullptr
 
     int64_t q_b, q_n, q_s;
     int64_t k_b, k_n, k_s;
     int64_t v_b, v_n, v_s;
     int64_t o_b, o_n, o_s;
+    int64_t qr_b, qr_n, qr_s;
+    int64_t kr_b, kr_n, kr_s;
     int64_t st_b, st_n, st_s;       // statistics; the 8 lanes are contiguous
     int64_t pse_b, pse_n, pse_i;    // dense bias strides (column stride 1); ALiBi: pse_b, pse_n
     int64_t mask_b, mask_n, mask_i; // mask strides (column stride 1), broadcast dims have 0
@@ -34,6 +38,7 @@ struct FaParams {
 
     int32_t B, Nq, Nkv, group;  // group = Nq / Nkv
     int32_t D, Dv;
+    int32_t Dr;                 // rope head dim (0 without queryRope/keyRope): S = Q K^T + Qr Kr^T
     int32_t Sq, Skv;            // sequence lengths (TND: the longest)
     int32_t pre, next;          // band, clamped to +-(Sq + Skv + 1)
     float scale;                // scaleValue in fp32
@@ -134,18 +139,22 @@ enum KernelKind { KERNEL_SIMT = 0, KERNEL_SM100 = 1 };
 struct alignas(64) TmaDesc {
     uint64_t opaque[16];
 };
+// Q, K, V and (with rope) queryRope, keyRope; without rope qr/kr repeat q/k
+// and are never read.
+struct TmaSet {
+    TmaDesc q, k, v, qr, kr;
+};
 
 cudaError_t launch_simt(const FaParams& p, cudaStream_t stream);
-cudaError_t launch_sm100(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk,
-                         const TmaDesc& tv, int num_sms, cudaStream_t stream);
+cudaError_t launch_sm100(const FaParams& p, const TmaSet& maps, int num_sms, cudaStream_t stream);
 // Schedule of the tcgen05 kernel (fills grid, n_whole, n_pieces, n_tickets
 // from n_items): one CTA per SM, and, when every work item costs the same
 // (`uniform`, item_kv_blocks 128-key blocks each) and the last wave is short,
 // the last wave's items split into key pieces.  Returns the bytes of partial
 // results the split needs (0 without a split).
 uint64_t plan_sm100_schedule(FaParams& p, int num_sms, bool uniform, int item_kv_blocks);
-// Encodes the Q/K/V tensor maps for the tcgen05 kernel.
-cudaError_t make_sm100_tmaps(const FaParams& p, TmaDesc* tq, TmaDesc* tk, TmaDesc* tv);
+// Encodes the Q/K/V (and rope) tensor maps for the tcgen05 kernel.
+cudaError_t make_sm100_tmaps(const FaParams& p, TmaSet* maps);
 uint64_t read_and_clear_device_error(cudaError_t* err);
 
 }  // namespace fa

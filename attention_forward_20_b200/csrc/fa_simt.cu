@@ -82,7 +82,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) fa_fwd_simt_kernel(const FaPar
     const T* Q = static_cast<const T*>(p.q) + b * p.q_b + n * p.q_n;
     const T* K = static_cast<const T*>(p.k) + b * p.k_b + nk * p.k_n;
     const T* V = static_cast<const T*>(p.v) + b * p.v_b + nk * p.v_n;
-    const int D = p.D, Dv = p.Dv;
+    // queryRope / keyRope: columns D .. D+Dr-1 of the dot product
+    const T* QR = p.Dr ? static_cast<const T*>(p.qr) + b * p.qr_b + n * p.qr_n : nullptr;
+    const T* KR = p.Dr ? static_cast<const T*>(p.kr) + b * p.kr_b + nk * p.kr_n : nullptr;
+    const int D = p.D, Dv = p.Dv, Dqk = p.D + p.Dr;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int i = i0 + warp;  // this warp's query row
     const bool row_ok = i < q_len;
@@ -90,7 +93,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) fa_fwd_simt_kernel(const FaPar
     // Q rows, zero-padded to DMAX (the dot products run over DMAX)
     for (int idx = tid; idx < kRows * DMAX; idx += blockDim.x) {
         const int r = idx / DMAX, d = idx % DMAX, ii = i0 + r;
-        sQ[r * ld + d] = (ii < q_len && d < D) ? to_f(Q[(q_off + ii) * p.q_s + d]) : 0.f;
+        float x = 0.f;
+        if (ii < q_len && d < D) x = to_f(Q[(q_off + ii) * p.q_s + d]);
+        else if (ii < q_len && d < Dqk) x = to_f(QR[(q_off + ii) * p.qr_s + (d - D)]);
+        sQ[r * ld + d] = x;
     }
 
     float slope = 0.f;
@@ -126,7 +132,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) fa_fwd_simt_kernel(const FaPar
                 const int idx = tid + (u + e) * (kWarps * 32);
                 const int r = idx / DMAX, d = idx % DMAX, j = j0 + r;
                 const bool in = j < kv_len;
-                kk[e] = (in && d < D) ? to_f(K[(kv_off + j) * p.k_s + d]) : 0.f;
+                kk[e] = (in && d < D) ? to_f(K[(kv_off + j) * p.k_s + d])
+                        : (in && d < Dqk) ? to_f(KR[(kv_off + j) * p.kr_s + (d - D)]) : 0.f;
                 vv[e] = (in && d < Dv) ? to_f(V[(kv_off + j) * p.v_s + d]) : 0.f;
             }
 #pragma unroll
@@ -232,7 +239,8 @@ cudaError_t launch_t(const FaParams& p, cudaStream_t stream) {
 
 template <typename T>
 cudaError_t launch_d(const FaParams& p, cudaStream_t stream) {
-    const int dmax = p.D > p.Dv ? p.D : p.Dv;
+    const int dqk = p.D + p.Dr;
+    const int dmax = dqk > p.Dv ? dqk : p.Dv;
     if (dmax <= 64) return launch_t<T, 64>(p, stream);
     if (dmax <= 128) return launch_t<T, 128>(p, stream);
     return launch_t<T, 256>(p, stream);

@@ -74,20 +74,28 @@ enum : int {
     kSiteSFull, kSiteOFull, kSiteDrain, kSiteInjected, kSiteSched
 };
 
-template <int D>
+// kRope: queryRope/keyRope with a head dim of 64 — one 128-byte chunk more
+// in every Q tile (after its D columns) and, for K, in a two-slot ring of
+// its own that fills with K under K's barrier.
+template <int D, bool kRope = false>
 struct Cfg {
     static constexpr int kChunks = D / 64;             // 128-byte swizzle chunks per row
     static constexpr int kChunkBytes = kTileM * 128;   // one chunk of a 128-row tile
-    static constexpr int kTileBytes = kTileM * D * 2;  // one Q, K or V tile
-    static constexpr int kStages = (D == 128) ? 4 : 8; // K/V ring slots
-    static constexpr int kSmemBytes = (2 + kStages) * kTileBytes + 1024;
+    static constexpr int kTileBytes = kTileM * D * 2;  // one K or V tile
+    static constexpr int kQTileBytes = kTileBytes + (kRope ? kChunkBytes : 0);
+    static constexpr int kRopeSlots = kRope ? 2 : 0;
+    static constexpr int kStages = (D == 128) ? (kRope ? 3 : 4) : 8;  // K/V ring slots
+    static constexpr int kSmemBytes = 2 * kQTileBytes + kStages * kTileBytes + kRopeSlots * kChunkBytes + 1024;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kOCol = 256;
 };
+static_assert(Cfg<128, true>::kSmemBytes + 1024 <= 227 * 1024, "rope tiles exceed shared memory");
+static_assert(Cfg<64, true>::kSmemBytes + 1024 <= 227 * 1024, "rope tiles exceed shared memory");
 
 struct Barriers {
     uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2];
     uint64_t kv_full[8], kv_empty[8];
+    uint64_t kr_empty[2];  // keyRope slots (the K load's kv_full also covers its keyRope chunk)
     uint64_t sched_full[kSched], sched_empty[kSched];
     uint64_t drain;
     uint64_t never;  // failure injection: initialised, never arrived on
@@ -263,24 +271,25 @@ __device__ __forceinline__ int take_ticket_local(const FaParams& p, Barriers& ba
 // TMA producer (one warp: every lane follows the schedule and waits, so all
 // operands stay warp-uniform; one elected lane issues the copies)
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool kRope>
 __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
-                             const CUtensorMap* tv, uint8_t* sQ, uint8_t* sKV, Barriers& bars,
-                             TicketSlots& slots, volatile int* abort) {
-    using C = Cfg<D>;
-    uint32_t kv_fill = 0, q_fill[2] = {0, 0}, k_sched = 0;
+                             const CUtensorMap* tv, const CUtensorMap* tqr, const CUtensorMap* tkr, uint8_t* sQ,
+                             uint8_t* sKV, uint8_t* sKr, Barriers& bars, TicketSlots& slots, volatile int* abort) {
+    using C = Cfg<D, kRope>;
+    uint32_t kv_fill = 0, q_fill[2] = {0, 0}, k_sched = 0, kr_fill = 0;
     bool ok = true;
 
-    auto load_tile = [&](const CUtensorMap* tm, uint8_t* dst, uint64_t* bar, int row, int head, int b,
-                         int64_t seq_off) {
-#pragma unroll
-        for (int c = 0; c < C::kChunks; ++c) {
+    auto load_chunks = [&](const CUtensorMap* tm, uint8_t* dst, uint64_t* bar, int chunks, int row, int head,
+                           int b, int64_t seq_off) {
+        for (int c = 0; c < chunks; ++c) {
             if (p.varlen)
                 tma_load_3d(dst + c * C::kChunkBytes, tm, bar, c * 64, (int)(seq_off + row), head);
             else
                 tma_load_4d(dst + c * C::kChunkBytes, tm, bar, c * 64, row, head, b);
         }
     };
+    auto load_tile = [&](const CUtensorMap* tm, uint8_t* dst, uint64_t* bar, int row, int head, int b,
+                         int64_t seq_off) { load_chunks(tm, dst, bar, C::kChunks, row, head, b, seq_off); };
 
     while (ok) {
         Item tit;
@@ -297,33 +306,44 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
         auto load_q = [&](int t) -> bool {
             if (!warp_wait(&bars.q_empty[t], (q_fill[t] & 1) ^ 1, abort, kSiteQEmpty)) return false;
             if (elect_one()) {
-                mbar_arrive_expect_tx(&bars.q_full[t], C::kTileBytes);
-                load_tile(tq, sQ + t * C::kTileBytes, &bars.q_full[t], it.qb * kQBlock + t * kTileM, it.n, it.b,
+                mbar_arrive_expect_tx(&bars.q_full[t], C::kQTileBytes);
+                load_tile(tq, sQ + t * C::kQTileBytes, &bars.q_full[t], it.qb * kQBlock + t * kTileM, it.n, it.b,
                           it.q_off);
+                if constexpr (kRope)
+                    load_chunks(tqr, sQ + t * C::kQTileBytes + C::kTileBytes, &bars.q_full[t], 1,
+                                it.qb * kQBlock + t * kTileM, it.n, it.b, it.q_off);
             }
             __syncwarp();
             ++q_fill[t];
             return true;
         };
-        auto load_kv = [&](const CUtensorMap* tm, int jb) -> bool {
+        auto load_kv = [&](const CUtensorMap* tm, int jb, bool with_rope) -> bool {
             const int slot = kv_fill % C::kStages;
             if (!warp_wait(&bars.kv_empty[slot], ((kv_fill / C::kStages) & 1) ^ 1, abort, kSiteKvEmpty))
                 return false;
+            const uint32_t rs = kr_fill % 2;
+            if (kRope && with_rope &&
+                !warp_wait(&bars.kr_empty[rs], ((kr_fill / 2) & 1) ^ 1, abort, kSiteKvEmpty))
+                return false;
             if (elect_one()) {
-                mbar_arrive_expect_tx(&bars.kv_full[slot], C::kTileBytes);
+                mbar_arrive_expect_tx(&bars.kv_full[slot], C::kTileBytes + (kRope && with_rope ? C::kChunkBytes : 0));
                 load_tile(tm, sKV + slot * C::kTileBytes, &bars.kv_full[slot], jb * kTileN, it.nk, it.b,
                           it.kv_off);
+                if (kRope && with_rope)
+                    load_chunks(tkr, sKr + rs * C::kChunkBytes, &bars.kv_full[slot], 1, jb * kTileN, it.nk, it.b,
+                                it.kv_off);
             }
             __syncwarp();
             ++kv_fill;
+            if (kRope && with_rope) ++kr_fill;
             return true;
         };
 
         if (tr[0].active() && !load_q(0)) { ok = false; break; }
         for (int jb = lo; ok && jb <= hi; ++jb) {
-            if (!load_kv(tk, jb)) { ok = false; break; }
+            if (!load_kv(tk, jb, true)) { ok = false; break; }
             if (jb == lo && tr[1].active() && !load_q(1)) { ok = false; break; }
-            if (!load_kv(tv, jb)) { ok = false; break; }
+            if (!load_kv(tv, jb, false)) { ok = false; break; }
         }
     }
 
@@ -345,14 +365,14 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
 // warp-uniform values; one elected lane issues each tcgen05 instruction, the
 // same lane every time, so its commits cover its MMAs)
 // ---------------------------------------------------------------------------
-template <typename T, int D>
-__device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& bars, const TicketSlots& slots,
-                        uint32_t tmem, volatile int* abort) {
-    using C = Cfg<D>;
+template <typename T, int D, bool kRope>
+__device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* sKr, Barriers& bars,
+                        const TicketSlots& slots, uint32_t tmem, volatile int* abort) {
+    using C = Cfg<D, kRope>;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     const uint32_t idesc_qk = idesc_f16(kBf16, kTileM, kTileN, false, false, p.neg_scale != 0);
     constexpr uint32_t idesc_pv = idesc_f16(kBf16, kTileM, D, false, true, false);
-    uint32_t kv_use = 0, q_use[2] = {0, 0}, p_cnt[2] = {0, 0}, k_sched = 0;
+    uint32_t kv_use = 0, q_use[2] = {0, 0}, p_cnt[2] = {0, 0}, k_sched = 0, kr_use = 0;
     bool ok = true;
     // Failure injection: a wait that can only end by running out of time.
     if (p.debug_stall && !warp_wait(&bars.never, 0, abort, kSiteInjected)) ok = false;
@@ -371,14 +391,21 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
     // swizzled, 8-row groups 1024 bytes apart, 64-column chunks one tile-chunk apart.
     // S_t = Q_t · K^T over D/16 K-steps, O_t (+)= P_t · V over 8 K-steps:
     // each group is one asm block issued by one elected lane.
-    auto issue_qk = [&](int t, int slot) {
-        const uint64_t qd = sdesc_sw128(smem_u32(sQ + t * C::kTileBytes), 1024, 16);
+    // With rope, 4 more K-steps over the queryRope / keyRope chunks accumulate
+    // into the same S.
+    auto issue_qk = [&](int t, int slot, uint32_t rs) {
+        const uint64_t qd = sdesc_sw128(smem_u32(sQ + t * C::kQTileBytes), 1024, 16);
         const uint64_t kd = sdesc_sw128(smem_u32(sKV + slot * C::kTileBytes), 1024, 16);
         if (elect_one()) {
             if constexpr (D == 128)
                 mma_ss_k128(tmem + t * kTileN, qd, kd, idesc_qk, 0u);
             else
                 mma_ss_k64(tmem + t * kTileN, qd, kd, idesc_qk, 0u);
+            if constexpr (kRope) {
+                const uint64_t qrd = sdesc_sw128(smem_u32(sQ + t * C::kQTileBytes + C::kTileBytes), 1024, 16);
+                const uint64_t krd = sdesc_sw128(smem_u32(sKr + rs * C::kChunkBytes), 1024, 16);
+                mma_ss_k64(tmem + t * kTileN, qrd, krd, idesc_qk, 1u);
+            }
         }
         __syncwarp();
     };
@@ -404,20 +431,23 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
         int sk;
         if (!ok || !wait_kv(&sk)) { ok = false; break; }
         tc_fence_after();
+        uint32_t rs = kr_use % 2;
         for (int t = 0; t < 2; ++t) {
             if (tr[t].has(lo)) {
-                issue_qk(t, sk);
+                issue_qk(t, sk, rs);
                 commit(&bars.s_full[t]);
                 if (lo == tr[t].hi) commit(&bars.q_empty[t]);
             }
         }
         commit(&bars.kv_empty[sk]);
+        if constexpr (kRope) { commit(&bars.kr_empty[rs]); ++kr_use; }
 
         for (int jb = lo; jb <= hi; ++jb) {
             int sv, sk2 = 0;
             const bool has_next = jb < hi;
             if (!wait_kv(&sv) || (has_next && !wait_kv(&sk2))) { ok = false; break; }
             tc_fence_after();
+            rs = kr_use % 2;
             for (int t = 0; t < 2; ++t) {
                 if (tr[t].has(jb)) {
                     if (!warp_wait(&bars.p_full[t], p_cnt[t] & 1, abort, kSitePFull)) { ok = false; break; }
@@ -427,7 +457,7 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
                     if (jb == tr[t].hi) commit(&bars.o_full[t]);
                 }
                 if (has_next && tr[t].has(jb + 1)) {
-                    issue_qk(t, sk2);
+                    issue_qk(t, sk2, rs);
                     commit(&bars.s_full[t]);
                     if (jb + 1 == tr[t].hi) commit(&bars.q_empty[t]);
                 }
@@ -435,6 +465,7 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& 
             if (!ok) break;
             commit(&bars.kv_empty[sv]);
             if (has_next) commit(&bars.kv_empty[sk2]);
+            if (kRope && has_next) { commit(&bars.kr_empty[rs]); ++kr_use; }
         }
         for (int t = 0; t < 2; ++t)
             if (tr[t].active()) ++q_use[t];
@@ -885,15 +916,17 @@ __global__ void __launch_bounds__(kMergeThreads) fa_merge_kernel(const FaParams 
 // ---------------------------------------------------------------------------
 // Kernel
 // ---------------------------------------------------------------------------
-template <typename T, int D, int kBias>
+template <typename T, int D, int kBias, bool kRope>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                        const __grid_constant__ CUtensorMap tmap_v, const FaParams p) {
-    using C = Cfg<D>;
+                        const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_qr,
+                        const __grid_constant__ CUtensorMap tmap_kr, const FaParams p) {
+    using C = Cfg<D, kRope>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
-    uint8_t* sKV = smem + 2 * C::kTileBytes;
+    uint8_t* sKV = smem + 2 * C::kQTileBytes;
+    uint8_t* sKr = sKV + C::kStages * C::kTileBytes;
     __shared__ Barriers bars;
     __shared__ TicketSlots slots;
     __shared__ uint32_t tmem_base;
@@ -912,6 +945,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars.kv_full[s], 1);
             mbar_init(&bars.kv_empty[s], 1);
         }
+        for (int r = 0; r < 2; ++r) mbar_init(&bars.kr_empty[r], 1);
         for (int k = 0; k < kSched; ++k) {
             mbar_init(&bars.sched_full[k], 1);
             mbar_init(&bars.sched_empty[k], kTicketReaders);
@@ -925,6 +959,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmap_q);
         prefetch_tmap(&tmap_k);
         prefetch_tmap(&tmap_v);
+        if (kRope) {
+            prefetch_tmap(&tmap_qr);
+            prefetch_tmap(&tmap_kr);
+        }
     }
     if (warp == kMmaWarp) {
         tmem_alloc(&tmem_base, C::kTmemCols);
@@ -941,9 +979,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         setmaxnreg_dec<kOtherRegs>();
         if (warp == kLoadWarp)
-            run_producer<D>(p, &tmap_q, &tmap_k, &tmap_v, sQ, sKV, bars, slots, &abort_flag);
+            run_producer<D, kRope>(p, &tmap_q, &tmap_k, &tmap_v, &tmap_qr, &tmap_kr, sQ, sKV, sKr, bars, slots,
+                                   &abort_flag);
         else if (warp == kMmaWarp)
-            run_mma<T, D>(p, sQ, sKV, bars, slots, tmem, &abort_flag);
+            run_mma<T, D, kRope>(p, sQ, sKV, sKr, bars, slots, tmem, &abort_flag);
     }
 
     tc_fence_before();
@@ -954,11 +993,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicCAS(&g_fa_error, 0ull, (static_cast<unsigned long long>(abort_flag) << 32) | (blockIdx.x + 1u));
 }
 
-template <typename T, int D, int kBias>
-cudaError_t launch_t(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, const TmaDesc& tv, int num_sms,
-                     cudaStream_t stream) {
-    using C = Cfg<D>;
-    auto kern = fa_fwd_sm100_kernel<T, D, kBias>;
+template <typename T, int D, int kBias, bool kRope = false>
+cudaError_t launch_t(const FaParams& p, const TmaSet& maps, int num_sms, cudaStream_t stream) {
+    using C = Cfg<D, kRope>;
+    auto kern = fa_fwd_sm100_kernel<T, D, kBias, kRope>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // setmaxnreg.inc can only hand out what the launch reserved: refuse to
@@ -971,9 +1009,9 @@ cudaError_t launch_t(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, co
         return cudaErrorLaunchOutOfResources;
     (void)num_sms;
     if (p.grid <= 0) return cudaSuccess;
-    kern<<<p.grid, kThreads, C::kSmemBytes, stream>>>(*reinterpret_cast<const CUtensorMap*>(&tq),
-                                                      *reinterpret_cast<const CUtensorMap*>(&tk),
-                                                      *reinterpret_cast<const CUtensorMap*>(&tv), p);
+    auto map = [](const TmaDesc& d) -> const CUtensorMap& { return *reinterpret_cast<const CUtensorMap*>(&d); };
+    kern<<<p.grid, kThreads, C::kSmemBytes, stream>>>(map(maps.q), map(maps.k), map(maps.v), map(maps.qr),
+                                                      map(maps.kr), p);
     e = cudaGetLastError();
     if (e != cudaSuccess || p.n_pieces == 0) return e;
     const int n_split = (p.n_tickets - p.n_whole) / p.n_pieces;
@@ -983,17 +1021,23 @@ cudaError_t launch_t(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, co
 }
 
 template <typename T>
-cudaError_t launch_d(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, const TmaDesc& tv, int num_sms,
-                     cudaStream_t stream) {
-    // pse_type is 0 whenever realShift is absent
-    if (p.D == 128) {
-        if (p.pse_type == 2) return launch_t<T, 128, 2>(p, tq, tk, tv, num_sms, stream);
-        if (p.pse_type == 1) return launch_t<T, 128, 1>(p, tq, tk, tv, num_sms, stream);
-        return launch_t<T, 128, 0>(p, tq, tk, tv, num_sms, stream);
+cudaError_t launch_d(const FaParams& p, const TmaSet& maps, int num_sms, cudaStream_t stream) {
+    // pse_type is 0 whenever realShift is absent; rope (bf16 only, no
+    // realShift) has kernels of its own
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        if (p.Dr) {
+            if (p.D == 128) return launch_t<T, 128, 0, true>(p, maps, num_sms, stream);
+            return launch_t<T, 64, 0, true>(p, maps, num_sms, stream);
+        }
     }
-    if (p.pse_type == 2) return launch_t<T, 64, 2>(p, tq, tk, tv, num_sms, stream);
-    if (p.pse_type == 1) return launch_t<T, 64, 1>(p, tq, tk, tv, num_sms, stream);
-    return launch_t<T, 64, 0>(p, tq, tk, tv, num_sms, stream);
+    if (p.D == 128) {
+        if (p.pse_type == 2) return launch_t<T, 128, 2>(p, maps, num_sms, stream);
+        if (p.pse_type == 1) return launch_t<T, 128, 1>(p, maps, num_sms, stream);
+        return launch_t<T, 128, 0>(p, maps, num_sms, stream);
+    }
+    if (p.pse_type == 2) return launch_t<T, 64, 2>(p, maps, num_sms, stream);
+    if (p.pse_type == 1) return launch_t<T, 64, 1>(p, maps, num_sms, stream);
+    return launch_t<T, 64, 0>(p, maps, num_sms, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -1025,14 +1069,14 @@ cuuint64_t stride_bytes(int64_t elems, int64_t size) {
 
 // Box of 64 columns (128 bytes, the swizzle span) x 128 rows; 128-byte swizzle;
 // out-of-range rows read as zero.
-cudaError_t encode(TmaDesc* out, const FaParams& p, const void* base, int rows, int heads, int64_t s_stride,
-                   int64_t n_stride, int64_t b_stride) {
+cudaError_t encode(TmaDesc* out, const FaParams& p, const void* base, int cols, int rows, int heads,
+                   int64_t s_stride, int64_t n_stride, int64_t b_stride) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
     const CUtensorMapDataType dt = p.dtype == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUresult r;
     if (p.varlen) {
-        const cuuint64_t dims[3] = {(cuuint64_t)p.D, (cuuint64_t)rows, (cuuint64_t)heads};
+        const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)heads};
         const cuuint64_t strides[2] = {stride_bytes(s_stride, rows), stride_bytes(n_stride, heads)};
         const cuuint32_t box[3] = {64, 128, 1};
         const cuuint32_t es[3] = {1, 1, 1};
@@ -1040,7 +1084,7 @@ cudaError_t encode(TmaDesc* out, const FaParams& p, const void* base, int rows, 
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     } else {
-        const cuuint64_t dims[4] = {(cuuint64_t)p.D, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)p.B};
+        const cuuint64_t dims[4] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)p.B};
         const cuuint64_t strides[3] = {stride_bytes(s_stride, rows), stride_bytes(n_stride, heads),
                                        stride_bytes(b_stride, p.B)};
         const cuuint32_t box[4] = {64, 128, 1, 1};
@@ -1054,10 +1098,18 @@ cudaError_t encode(TmaDesc* out, const FaParams& p, const void* base, int rows, 
 
 }  // namespace
 
-cudaError_t make_sm100_tmaps(const FaParams& p, TmaDesc* tq, TmaDesc* tk, TmaDesc* tv) {
-    cudaError_t e = encode(tq, p, p.q, p.Tq, p.Nq, p.q_s, p.q_n, p.q_b);
-    if (e == cudaSuccess) e = encode(tk, p, p.k, p.Tkv, p.Nkv, p.k_s, p.k_n, p.k_b);
-    if (e == cudaSuccess) e = encode(tv, p, p.v, p.Tkv, p.Nkv, p.v_s, p.v_n, p.v_b);
+cudaError_t make_sm100_tmaps(const FaParams& p, TmaSet* maps) {
+    cudaError_t e = encode(&maps->q, p, p.q, p.D, p.Tq, p.Nq, p.q_s, p.q_n, p.q_b);
+    if (e == cudaSuccess) e = encode(&maps->k, p, p.k, p.D, p.Tkv, p.Nkv, p.k_s, p.k_n, p.k_b);
+    if (e == cudaSuccess) e = encode(&maps->v, p, p.v, p.D, p.Tkv, p.Nkv, p.v_s, p.v_n, p.v_b);
+    if (e != cudaSuccess) return e;
+    if (p.Dr) {
+        e = encode(&maps->qr, p, p.qr, p.Dr, p.Tq, p.Nq, p.qr_s, p.qr_n, p.qr_b);
+        if (e == cudaSuccess) e = encode(&maps->kr, p, p.kr, p.Dr, p.Tkv, p.Nkv, p.kr_s, p.kr_n, p.kr_b);
+    } else {
+        maps->qr = maps->q;
+        maps->kr = maps->k;
+    }
     return e;
 }
 
@@ -1080,10 +1132,9 @@ uint64_t plan_sm100_schedule(FaParams& p, int num_sms, bool uniform, int item_kv
     return static_cast<uint64_t>(tail) * pieces * kQBlock * (p.D + 4) * sizeof(float);
 }
 
-cudaError_t launch_sm100(const FaParams& p, const TmaDesc& tq, const TmaDesc& tk, const TmaDesc& tv, int num_sms,
-                         cudaStream_t stream) {
-    if (p.dtype == 2) return launch_d<__nv_bfloat16>(p, tq, tk, tv, num_sms, stream);
-    return launch_d<__half>(p, tq, tk, tv, num_sms, stream);
+cudaError_t launch_sm100(const FaParams& p, const TmaSet& maps, int num_sms, cudaStream_t stream) {
+    if (p.dtype == 2) return launch_d<__nv_bfloat16>(p, maps, num_sms, stream);
+    return launch_d<__half>(p, maps, num_sms, stream);
 }
 
 uint64_t read_and_clear_device_error(cudaError_t* err) {

@@ -241,9 +241,9 @@ extern "C" fa_status fa_fwd_varlen_static(
             return FA_ERR_CUDA;
         fa::plan_sm100_schedule(p, sms, false, 0);  // varlen items differ in cost: no split
         p.sched_counter = reinterpret_cast<int*>(dev);
-        fa::TmaDesc tq, tk, tv;
-        if (fa::make_sm100_tmaps(p, &tq, &tk, &tv) != cudaSuccess) return FA_ERR_CUDA;
-        err = fa::launch_sm100(p, tq, tk, tv, p.grid, st);
+        fa::TmaSet maps;
+        if (fa::make_sm100_tmaps(p, &maps) != cudaSuccess) return FA_ERR_CUDA;
+        err = fa::launch_sm100(p, maps, p.grid, st);
     } else {
         err = fa::launch_simt(p, st);
     }

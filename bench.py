@@ -27,7 +27,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from workloads import build  # noqa: E402
+from workloads import build, normal  # noqa: E402
 
 METRIC = "FA forward TFLOP/s and % of B200 dense BF16/FP16 peak (1 GPU)"
 UNIT = "TFLOP/s"
@@ -199,6 +199,16 @@ def alibi_bias_on_device(slopes, seq, first_row, dtype, dev):
     return bias
 
 
+def rope_tensors(w, dr, seed):
+    """queryRope / keyRope for workload w: the query's / key's layout and sizes, head dim dr."""
+    def shaped(t, heads):
+        if w.layout in ("BSH", "SBH"):
+            return tuple(t.shape[:2]) + (heads * dr,)
+        return tuple(t.shape[:-1]) + (dr,)
+    n_kv = w.k.shape[-1] // (w.q.shape[-1] // w.head_num) if w.layout in ("BSH", "SBH") else None
+    return (normal(shaped(w.q, w.head_num), "bf16", seed), normal(shaped(w.k, n_kv), "bf16", seed + 1))
+
+
 def fa_kwargs(w, dev):
     c = lambda t: None if t is None else t.to(dev)  # noqa: E731
     pse = c(w.pse)
@@ -209,11 +219,17 @@ def fa_kwargs(w, dev):
                 softmax_out_layout=w.softmax_out_layout)
 
 
-def time_oracle(w, budget_s, max_heads=None):
+def time_oracle(w, budget_s, max_heads=None, rope=None):
     """Float64 oracle on whole (batch, head) pairs of the workload until
-    `budget_s` seconds have passed; returns (flops done, seconds, heads done)."""
+    `budget_s` seconds have passed; returns (flops done, seconds, heads done).
+    rope: (queryRope, keyRope) host tensors or None."""
     from oracle import ref
     d = w.q.shape[-1] if w.layout not in ("BSH", "SBH") else w.q.shape[-1] // w.head_num
+    dr = 0
+    if rope is not None:
+        dr = rope[0].shape[-1] if w.layout not in ("BSH", "SBH") else rope[0].shape[-1] // w.head_num
+        qrh = ref.heads_view(rope[0].double().numpy(), w.layout, dr)
+        krh = ref.heads_view(rope[1].double().numpy(), w.layout, dr)
     qh = ref.heads_view(w.q.double().numpy(), w.layout, d)
     kh = ref.heads_view(w.k.double().numpy(), w.layout, d)
     vh = ref.heads_view(w.v.double().numpy(), w.layout, d)
@@ -230,18 +246,23 @@ def time_oracle(w, budget_s, max_heads=None):
     flops = secs = 0.0
     heads = 0
     for (b, n) in pairs[:max_heads]:
+        qr = kr = None
         if w.layout == "TND":
             q, k, v = (qh[cq[b]:cq[b + 1], n], kh[ck[b]:ck[b + 1], n // group], vh[ck[b]:ck[b + 1], n // group])
+            if dr:
+                qr, kr = qrh[cq[b]:cq[b + 1], n], krh[ck[b]:ck[b + 1], n // group]
         else:
             q, k, v = qh[b, n], kh[b, n // group], vh[b, n // group]
+            if dr:
+                qr, kr = qrh[b, n], krh[b, n // group]
         rows = np.arange(q.shape[0])
         t0 = time.perf_counter()
         ref.head_forward(q, k, v, w.scale, rows=rows,
                          pse=ref._pse_rows(pse, w.pse_type, b, n, rows, k.shape[0]),
                          pre_tokens=w.pre_tokens, next_tokens=w.next_tokens,
-                         sink=None if sink is None else sink[n])
+                         sink=None if sink is None else sink[n], q_rope=qr, k_rope=kr)
         secs += time.perf_counter() - t0
-        flops += 4.0 * d * q.shape[0] * k.shape[0]
+        flops += (4.0 * d + 2.0 * dr) * q.shape[0] * k.shape[0]
         heads += 1
         if secs >= budget_s:
             break
@@ -334,6 +355,8 @@ def main():
                          "then fa_lse_merge (dense layouts)")
     ap.add_argument("--pse", default="slopes", choices=["slopes", "dense", "compressed"],
                     help="ALiBi workloads: slopes in-kernel, a materialised [1,N,S,S] bias, or its last 1024 rows")
+    ap.add_argument("--rope", type=int, default=0,
+                    help="bf16 workloads: add queryRope/keyRope of this head dim (N(0,1), seeded)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -358,6 +381,16 @@ def main():
     flops_tiles, flops_exact = tile_flops(w)
     q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
     kw = fa_kwargs(w, dev)
+    rope = None
+    if args.rope:
+        if w.dtype != "bf16":
+            raise SystemExit("--rope needs a bf16 workload (queryRope/keyRope are BFLOAT16 only)")
+        rope = rope_tensors(w, args.rope, seed=9100 + rank)
+        kw["query_rope"], kw["key_rope"] = rope[0].to(dev), rope[1].to(dev)
+        # S = Q K^T + Qr Kr^T: 2*(D + Dr) + 2*Dv FLOPs per kept pair instead of 4*D
+        d = w.q.shape[-1] // w.head_num if w.layout in ("BSH", "SBH") else w.q.shape[-1]
+        flops_tiles *= (4.0 * d + 2.0 * args.rope) / (4.0 * d)
+        flops_exact *= (4.0 * d + 2.0 * args.rope) / (4.0 * d)
     bias_bytes = 0
     if args.pse != "slopes" and w.pse_type == 2:
         # the same ALiBi bias, materialised in the query dtype and resident in HBM
@@ -440,17 +473,19 @@ def main():
         raise SystemExit(f"kernel error word {word:#x}")
 
     # end to end: pinned host inputs -> device, forward, result -> pinned host
-    host = [t.pin_memory() for t in (w.q, w.k, w.v)]
+    host = [t.pin_memory() for t in (w.q, w.k, w.v) + (tuple(rope) if rope is not None else ())]
     host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     host_sm = torch.empty(smax.shape, dtype=smax.dtype).pin_memory()
     host_ss = torch.empty(ssum.shape, dtype=ssum.dtype).pin_memory()
-    dq, dk, dv = (torch.empty_like(t, device=dev) for t in host)
+    dev_in = [torch.empty_like(t, device=dev) for t in host]
+    dq, dk, dv = dev_in[:3]
+    kw_e2e = dict(kw, **({"query_rope": dev_in[3], "key_rope": dev_in[4]} if rope is not None else {}))
     e2e_steps = max(3, min(args.steps, 20))
 
     def e2e_step():
-        for d_, h_ in zip((dq, dk, dv), host):
+        for d_, h_ in zip(dev_in, host):
             d_.copy_(h_, non_blocking=True)
-        fa.fa_fwd(dq, dk, dv, out=out, softmax_max=smax, softmax_sum=ssum, **kw)
+        fa.fa_fwd(dq, dk, dv, out=out, softmax_max=smax, softmax_sum=ssum, **kw_e2e)
         host_out.copy_(out, non_blocking=True)
         host_sm.copy_(smax, non_blocking=True)
         host_ss.copy_(ssum, non_blocking=True)
@@ -479,8 +514,8 @@ def main():
     value = whole_job_tflops(flops_tiles, world, ms_per_step)
     per_gpu = flops_tiles / (ms_per_step * 1e-3) / 1e12
     peak, peak_src = load_peak()
-    traffic = load_traffic(w.name) if args.pse == "slopes" else None
-    fl, secs, heads = time_oracle(w, args.cpu_budget)
+    traffic = load_traffic(w.name) if args.pse == "slopes" and not args.rope else None
+    fl, secs, heads = time_oracle(w, args.cpu_budget, rope=rope)
     cpu_value = fl / secs / 1e12
     desc = workload_desc(w)
     merge_line = None
@@ -491,6 +526,8 @@ def main():
         part_bytes = out.numel() * out.element_size() + 2 * smax.numel() * smax.element_size()
         merge_line = hbm_line(0, q, k, v, out, merge_ms, bytes_override=(args.kv_chunks + 1) * part_bytes)
         merge_line["ms"] = merge_ms
+    if rope is not None:
+        desc["rope"] = f"queryRope/keyRope head dim {args.rope} (bf16, N(0,1)): S = scale*(Q K^T + Qr Kr^T)"
     if args.pse != "slopes" and w.pse_type == 2:
         desc["pse"] = ("materialised fp16 bias [1,N,S,S], resident" if args.pse == "dense"
                        else "compressed bias: last 1024 rows [1,N,1024,S], resident")

@@ -152,9 +152,20 @@ FA_API fa_status fa_fwd_get_workspace_size(
     const fa_tensor* softmaxMax, const fa_tensor* softmaxSum, const fa_tensor* attentionOut,
     uint64_t* workspaceSize, fa_executor** executor);
 
-/* Stage 1 with global positions (aclnnFlashAttentionVarLenScoreV5,
+/* Stage 1 with the rope term and global positions
+ * (aclnnFlashAttentionVarLenScoreV5GetWorkspaceSize's further arguments).
+ *
+ * queryRope / keyRope (optional, together; the page's forward formula
+ * scale*(query key^T + queryRope keyRope^T) + pse): BFLOAT16 tensors (query,
+ * key and value must then be BFLOAT16 too; else 161002) in inputLayout with
+ * the sizes and head counts of query / key and a head dim Dr of their own
+ * (BSH/SBH: H = heads * Dr); D + Dr <= 256.  Not with realShift (the page:
+ * incompatible), pseType 0 or 1.  A mismatch returns 561103.  Dr = 64 with
+ * D = Dv in {64, 128} runs on the tensor cores; other sizes on the CUDA-core
+ * kernel.
+ *
  * qStartIdxOptional / kvStartIdxOptional: the start, in the whole sequence, of
- * the query and key/value chunk this call sees).  The band and an ALiBi bias
+ * the query and key/value chunk this call sees.  The band and an ALiBi bias
  * are evaluated at global positions qStart + i and kvStart + j:
  *   keep iff -preTokens <= (kvStart + j) - (qStart + i) <= nextTokens,
  *   ALiBi pse = -slope * |(qStart + i) - (kvStart + j)|;
@@ -163,9 +174,11 @@ FA_API fa_status fa_fwd_get_workspace_size(
  * sequence (nQStartIdx / nKvStartIdx entries, "TND" only for more than one);
  * kvStart - qStart must be the same for every sequence (else 561103).  All
  * other arguments and the return values are those of
- * fa_fwd_get_workspace_size, which equals this call with both NULL. */
+ * fa_fwd_get_workspace_size, which equals this call with queryRope, keyRope,
+ * qStartIdx and kvStartIdx all NULL. */
 FA_API fa_status fa_fwd_get_workspace_size_v5(
-    const fa_tensor* query, const fa_tensor* key, const fa_tensor* value,
+    const fa_tensor* query, const fa_tensor* queryRope, const fa_tensor* key, const fa_tensor* keyRope,
+    const fa_tensor* value,
     const fa_tensor* realShift, const fa_tensor* attenMask, const fa_tensor* sink,
     const int64_t* actualSeqQLen, int64_t nSeqQ,
     const int64_t* actualSeqKvLen, int64_t nSeqKv,

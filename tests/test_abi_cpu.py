@@ -410,6 +410,45 @@ def test_plan_start_indices_shift_must_be_common():
     assert plan(q, k, v, kv_start_idx=-1, **base)[0] == _abi.FA_ERR_INNER_NULLPTR
 
 
+def test_plan_rope_routes_and_validates():
+    """queryRope / keyRope (aclnnFlashAttentionVarLenScoreV5 parameter list):
+    bf16 only, both together, no realShift, the query's / key's sizes with a
+    head dim of their own."""
+    cum = [300, 500]
+    base = dict(input_layout="TND", head_num=4, actual_seq_qlen=cum, actual_seq_kvlen=cum, next_tokens=0)
+    q = torch.zeros(500, 4, 128, dtype=torch.bfloat16)
+    k = v = torch.zeros(500, 2, 128, dtype=torch.bfloat16)
+    qr = torch.zeros(500, 4, 64, dtype=torch.bfloat16)
+    kr = torch.zeros(500, 2, 64, dtype=torch.bfloat16)
+    st, _, text = plan(q, k, v, query_rope=qr, key_rope=kr, **base)
+    assert st == 0 and "kernel=sm100_tcgen05" in text and "Dr=64" in text
+    # another rope head dim: CUDA-core kernel
+    st, _, text = plan(q, k, v, query_rope=qr[..., :32], key_rope=kr[..., :32].contiguous(), **base)
+    assert st == 0 and "kernel=simt" in text and "Dr=32" in text
+    # one without the other, a realShift with it, wrong sizes or head counts
+    assert plan(q, k, v, query_rope=qr, **base)[0] == _abi.FA_ERR_INNER_NULLPTR
+    assert plan(q, k, v, key_rope=kr, **base)[0] == _abi.FA_ERR_INNER_NULLPTR
+    slopes = torch.ones(4)
+    assert plan(q, k, v, query_rope=qr, key_rope=kr, real_shift=slopes, pse_type=2,
+                **base)[0] == _abi.FA_ERR_INNER_NULLPTR
+    assert plan(q, k, v, query_rope=qr, key_rope=kr[..., :32].contiguous(), **base)[0] == _abi.FA_ERR_INNER_NULLPTR
+    assert plan(q, k, v, query_rope=qr[:499], key_rope=kr, **base)[0] == _abi.FA_ERR_INNER_NULLPTR
+    assert plan(q, k, v, query_rope=kr, key_rope=kr, **base)[0] == _abi.FA_ERR_INNER_NULLPTR
+    big = torch.zeros(500, 4, 192, dtype=torch.bfloat16)
+    bigk = torch.zeros(500, 2, 192, dtype=torch.bfloat16)
+    assert plan(q, k, v, query_rope=big, key_rope=bigk, **base)[0] == _abi.FA_ERR_INNER_NULLPTR  # D + Dr > 256
+    # dtypes: rope bf16 and query bf16
+    assert plan(q, k, v, query_rope=qr.half(), key_rope=kr.half(), **base)[0] == _abi.FA_ERR_PARAM_INVALID
+    qh, kh = q.half(), k.half()
+    assert plan(qh, kh, kh, query_rope=qr, key_rope=kr, **base)[0] == _abi.FA_ERR_PARAM_INVALID
+    # dense layouts: BSH rope has H = heads * Dr
+    qb = torch.zeros(2, 100, 4 * 64, dtype=torch.bfloat16)
+    kb = torch.zeros(2, 100, 2 * 64, dtype=torch.bfloat16)
+    st, _, text = plan(qb, kb, kb, input_layout="BSH", head_num=4, query_rope=torch.zeros(2, 100, 4 * 64,
+                       dtype=torch.bfloat16), key_rope=torch.zeros(2, 100, 2 * 64, dtype=torch.bfloat16))
+    assert st == 0 and "Dr=64" in text and "kernel=sm100_tcgen05" in text
+
+
 def _merge_status(outs, maxes, sums, out, smax, ssum, layout="BNSD", heads=2):
     lib = _abi.load()
     n = len(outs)

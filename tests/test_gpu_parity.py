@@ -435,3 +435,106 @@ def test_query_chunk_at_its_start(dtype, d):
     check_out(f64(out), want["out"][:, :, a:b], dtype)
     check_stats(f64(smax), want["softmax_max"][:, :, a:b], "softmaxMax")
     check_stats(f64(ssum), want["softmax_sum"][:, :, a:b], "softmaxSum")
+
+
+# ---------------------------------------------------------------------------
+# queryRope / keyRope: S = scale * (Q K^T + Qr Kr^T) (the V5 page's formula)
+# ---------------------------------------------------------------------------
+
+def _rope_case(layout, shape_q, shape_k, dr_shape_q, dr_shape_k, heads, seed, **kw):
+    w = W(layout, "bf16", shape_q, heads, seed, kshape=shape_k, **kw)
+    qr = normal(dr_shape_q, "bf16", seed + 10)
+    kr = normal(dr_shape_k, "bf16", seed + 11)
+    return w, qr, kr
+
+
+def _rope_compare(w, qr, kr, kernel):
+    q, k, v, pse, mask, sink = (None if t is None else t.cuda()
+                                for t in (w.q, w.k, w.v, w.pse, w.atten_mask, w.sink))
+    kw = dict(input_layout=w.layout, head_num=w.head_num, scale=w.scale, atten_mask=mask, sink=sink,
+              actual_seq_qlen=w.actual_seq_q, actual_seq_kvlen=w.actual_seq_kv, pre_tokens=w.pre_tokens,
+              next_tokens=w.next_tokens, query_rope=qr.cuda(), key_rope=kr.cuda())
+    assert kernel in fa.plan(q, k, v, **kw)[2]
+    out, smax, ssum = fa.fa_fwd(q, k, v, **kw)
+    torch.cuda.synchronize()
+    want = ref.forward(f64(w.q), f64(w.k), f64(w.v), layout=w.layout, head_num=w.head_num, scale=w.scale,
+                       atten_mask=f64(w.atten_mask), pre_tokens=w.pre_tokens, next_tokens=w.next_tokens,
+                       sink=f64(w.sink), actual_seq_q=w.actual_seq_q, actual_seq_kv=w.actual_seq_kv,
+                       query_rope=f64(qr), key_rope=f64(kr))
+    check_out(f64(out), want["out"], "bf16")
+    check_stats(f64(smax), want["softmax_max"], "softmaxMax")
+    check_stats(f64(ssum), want["softmax_sum"], "softmaxSum")
+
+
+from oracle import ref  # noqa: E402
+
+
+def test_rope_worked_example():
+    """The V5 page's call example, rope tensors included: T=256, N=1, D=128,
+    Dr=64, everything 1, uint8 mask of zeros, sink 3.0, scale 0.088388."""
+    t = 256
+    one = torch.ones(t, 1, 128, dtype=torch.bfloat16, device="cuda")
+    rope = torch.ones(t, 1, 64, dtype=torch.bfloat16, device="cuda")
+    out, smax, ssum = fa.fa_fwd(one, one, one, input_layout="TND", head_num=1, scale=0.088388,
+                                atten_mask=torch.zeros(t, t, dtype=torch.uint8, device="cuda"),
+                                sink=torch.tensor([3.0], device="cuda"), actual_seq_qlen=[t], actual_seq_kvlen=[t],
+                                pre_tokens=65536, next_tokens=65536, softmax_out_layout="same_as_input",
+                                query_rope=rope, key_rope=rope)
+    torch.cuda.synchronize()
+    m = 0.088388 * 192
+    assert out.float().eq(1.0).all()
+    assert smax.shape == (t, 1, 8)
+    check_stats(f64(smax), np.full((t, 1, 8), m), "softmaxMax")
+    check_stats(f64(ssum), np.full((t, 1, 8), t + np.exp(3.0 - m)), "softmaxSum")
+
+
+@pytest.mark.parametrize("case", ["tnd_gqa_causal_sink", "bnsd_d64", "bsh_band"])
+def test_rope_tcgen05(case):
+    if case == "tnd_gqa_causal_sink":
+        lens = [300, 0, 513, 129]
+        t = sum(lens)
+        w, qr, kr = _rope_case("TND", (t, 4, 128), (t, 2, 128), (t, 4, 64), (t, 2, 64), 4, 3700,
+                               actual_seq_q=cumulative(lens, False), actual_seq_kv=cumulative(lens, False),
+                               next_tokens=0, sink=normal((4,), "f32", 3720))
+    elif case == "bnsd_d64":
+        w, qr, kr = _rope_case("BNSD", (2, 3, 300, 64), (2, 3, 333, 64), (2, 3, 300, 64), (2, 3, 333, 64), 3, 3730)
+    else:
+        w, qr, kr = _rope_case("BSH", (2, 260, 2 * 128), (2, 260, 2 * 128), (2, 260, 2 * 64), (2, 260, 2 * 64), 2,
+                               3740, pre_tokens=100, next_tokens=20)
+    _rope_compare(w, qr, kr, "sm100_tcgen05")
+
+
+@pytest.mark.parametrize("d,dr", [(96, 32), (64, 128)])
+def test_rope_cuda_core_kernel(d, dr):
+    lens = [77, 190]
+    t = sum(lens)
+    w, qr, kr = _rope_case("TND", (t, 2, d), (t, 2, d), (t, 2, dr), (t, 2, dr), 2, 3750 + d,
+                           actual_seq_q=cumulative(lens, False), actual_seq_kv=cumulative(lens, False),
+                           next_tokens=0)
+    _rope_compare(w, qr, kr, "simt")
+
+
+def test_full_size_varlen_with_rope_sampled():
+    """The varlen causal bf16 workload at full size with Dr = 64 rope tensors,
+    in the bench's configuration (`bench.py --workload 4 --rope`); sampled rows."""
+    w = build(4)
+    t, nq = w.q.shape[0], w.head_num
+    nkv = w.k.shape[1]
+    qr, kr = normal((t, nq, 64), "bf16", 3800), normal((t, nkv, 64), "bf16", 3801)
+    q, k, v = w.q.cuda(), w.k.cuda(), w.v.cuda()
+    kw = dict(input_layout="TND", head_num=nq, scale=w.scale, actual_seq_qlen=w.actual_seq_q,
+              actual_seq_kvlen=w.actual_seq_kv, pre_tokens=w.pre_tokens, next_tokens=w.next_tokens,
+              softmax_out_layout=w.softmax_out_layout, query_rope=qr.cuda(), key_rope=kr.cuda())
+    assert "sm100_tcgen05" in fa.plan(q, k, v, **kw)[2]
+    res = fa.fa_fwd(q, k, v, **kw)
+    torch.cuda.synchronize()
+    rows = sample_rows(w, 48, seed=7)
+    from tests.parity import gather_rows
+    o, m, l = gather_rows(w, *res, rows)
+    wo, wm, wl = ref.forward_rows(f64(w.q), f64(w.k), f64(w.v), rows, layout="TND", head_num=nq, scale=w.scale,
+                                  pre_tokens=w.pre_tokens, next_tokens=w.next_tokens,
+                                  actual_seq_q=w.actual_seq_q, actual_seq_kv=w.actual_seq_kv,
+                                  query_rope=f64(qr), key_rope=f64(kr))
+    check_out(o, wo, "bf16", "sampled attentionOut rows")
+    check_stats(m, wm, "sampled softmaxMax")
+    check_stats(l, wl, "sampled softmaxSum")
