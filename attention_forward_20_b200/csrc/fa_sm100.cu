@@ -278,6 +278,7 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
     using C = Cfg<D, kRope>;
     uint32_t kv_fill = 0, q_fill[2] = {0, 0}, k_sched = 0, kr_fill = 0;
     bool ok = true;
+    const int v_chunks = (p.Dv + 63) / 64;
 
     auto load_chunks = [&](const CUtensorMap* tm, uint8_t* dst, uint64_t* bar, int chunks, int row, int head,
                            int b, int64_t seq_off) {
@@ -317,7 +318,11 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
             ++q_fill[t];
             return true;
         };
-        auto load_kv = [&](const CUtensorMap* tm, int jb, bool with_rope) -> bool {
+        // K tiles: all kChunks chunks (columns past D read as zero); V tiles:
+        // the chunks that hold its Dv columns.
+        auto load_kv = [&](const CUtensorMap* tm, int jb, bool is_k) -> bool {
+            const bool with_rope = is_k;
+            const int chunks = is_k ? C::kChunks : v_chunks;
             const int slot = kv_fill % C::kStages;
             if (!warp_wait(&bars.kv_empty[slot], ((kv_fill / C::kStages) & 1) ^ 1, abort, kSiteKvEmpty))
                 return false;
@@ -326,9 +331,10 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
                 !warp_wait(&bars.kr_empty[rs], ((kr_fill / 2) & 1) ^ 1, abort, kSiteKvEmpty))
                 return false;
             if (elect_one()) {
-                mbar_arrive_expect_tx(&bars.kv_full[slot], C::kTileBytes + (kRope && with_rope ? C::kChunkBytes : 0));
-                load_tile(tm, sKV + slot * C::kTileBytes, &bars.kv_full[slot], jb * kTileN, it.nk, it.b,
-                          it.kv_off);
+                mbar_arrive_expect_tx(&bars.kv_full[slot],
+                                      chunks * C::kChunkBytes + (kRope && with_rope ? C::kChunkBytes : 0));
+                load_chunks(tm, sKV + slot * C::kTileBytes, &bars.kv_full[slot], chunks, jb * kTileN, it.nk, it.b,
+                            it.kv_off);
                 if (kRope && with_rope)
                     load_chunks(tkr, sKr + rs * C::kChunkBytes, &bars.kv_full[slot], 1, jb * kTileN, it.nk, it.b,
                                 it.kv_off);
@@ -371,7 +377,8 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* s
     using C = Cfg<D, kRope>;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     const uint32_t idesc_qk = idesc_f16(kBf16, kTileM, kTileN, false, false, p.neg_scale != 0);
-    constexpr uint32_t idesc_pv = idesc_f16(kBf16, kTileM, D, false, true, false);
+    // P·V over the 64-column chunks that hold V's Dv columns
+    const uint32_t idesc_pv = idesc_f16(kBf16, kTileM, ((p.Dv + 63) / 64) * 64, false, true, false);
     uint32_t kv_use = 0, q_use[2] = {0, 0}, p_cnt[2] = {0, 0}, k_sched = 0, kr_use = 0;
     bool ok = true;
     // Failure injection: a wait that can only end by running out of time.
@@ -585,6 +592,28 @@ __device__ __forceinline__ void store_out32(const FaParams& p, T* orow, int cc, 
     }
 }
 
+// The first 8*groups (< 32) output columns from cc of a row: the last, partial
+// 32-column group of a value head dim that is a multiple of 8 only.
+template <typename T>
+__device__ __forceinline__ void store_out8s(const FaParams& p, T* orow, int cc, int groups, const uint32_t (&o)[32],
+                                            float o_scale) {
+#pragma unroll
+    for (int g = 0; g < 3; ++g) {
+        if (g >= groups) break;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            w[e] = pack2<T>(__uint_as_float(o[8 * g + 2 * e]) * o_scale, __uint_as_float(o[8 * g + 2 * e + 1]) * o_scale);
+        if (p.o_vec) {
+            *reinterpret_cast<uint4*>(orow + cc + 8 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+            const T* h = reinterpret_cast<const T*>(w);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) orow[cc + 8 * g + e] = h[e];
+        }
+    }
+}
+
 // softmaxMax (natural log units) and softmaxSum of query row i, all 8 lanes.
 __device__ __forceinline__ void store_stats(const FaParams& p, const Item& it, int i, const RowFinal& f) {
     const int64_t so = it.b * p.st_b + it.n * p.st_n + (it.q_off + i) * p.st_s;
@@ -789,6 +818,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                 // stable: the commit behind this block's S_t covered the last P·V.
 #pragma unroll
                 for (int cc = 0; cc < D; cc += 32) {
+                    if (cc >= p.Dv) break;
                     uint32_t o[32];
                     tmem_ld_x32(tO + cc, o);
 #pragma unroll
@@ -835,7 +865,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
         const RowFinal f = finalize_row(p, it, m_run, m_used, l);
         T* orow = static_cast<T*>(p.o) + it.b * p.o_b + it.n * p.o_n + (it.q_off + i) * p.o_s;
 #pragma unroll 1
-        for (int cc = 0; cc < D; cc += 32) {
+        for (int cc = 0; cc < p.Dv; cc += 32) {
             uint32_t o[32];
             if (has_blocks) {
                 tmem_ld_x32(tO + cc, o);
@@ -843,7 +873,11 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
 #pragma unroll
                 for (int e = 0; e < 32; ++e) o[e] = 0u;
             }
-            if (row_ok) store_out32<T>(p, orow, cc, o, f.o_scale);
+            if (!row_ok) continue;
+            if (cc + 32 <= p.Dv)
+                store_out32<T>(p, orow, cc, o, f.o_scale);
+            else
+                store_out8s<T>(p, orow, cc, (p.Dv - cc) / 8, o, f.o_scale);
         }
         if (row_ok) store_stats(p, it, i, f);
     }
@@ -862,6 +896,7 @@ __global__ void __launch_bounds__(kMergeThreads) fa_merge_kernel(const FaParams 
     const int idx = blockIdx.x * kMergeThreads + threadIdx.x;
     if (idx >= n_split * kQBlock * kGroups) return;
     const int g = idx % kGroups;
+    if (8 * g >= p.Dv) return;  // padding columns of a value head dim below D
     const int rr = idx / kGroups;
     const int r = rr % kQBlock, u = rr / kQBlock;
     const Item it = decode_item(p, p.n_whole + u);
@@ -1024,13 +1059,15 @@ template <typename T>
 cudaError_t launch_d(const FaParams& p, const TmaSet& maps, int num_sms, cudaStream_t stream) {
     // pse_type is 0 whenever realShift is absent; rope (bf16 only, no
     // realShift) has kernels of its own
+    // head dims up to 64 run on the 64-column kernels, up to 128 on the
+    // 128-column ones (columns past D and Dv load as zero)
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         if (p.Dr) {
-            if (p.D == 128) return launch_t<T, 128, 0, true>(p, maps, num_sms, stream);
+            if (p.D > 64) return launch_t<T, 128, 0, true>(p, maps, num_sms, stream);
             return launch_t<T, 64, 0, true>(p, maps, num_sms, stream);
         }
     }
-    if (p.D == 128) {
+    if (p.D > 64) {
         if (p.pse_type == 2) return launch_t<T, 128, 2>(p, maps, num_sms, stream);
         if (p.pse_type == 1) return launch_t<T, 128, 1>(p, maps, num_sms, stream);
         return launch_t<T, 128, 0>(p, maps, num_sms, stream);
@@ -1068,7 +1105,8 @@ cuuint64_t stride_bytes(int64_t elems, int64_t size) {
 }
 
 // Box of 64 columns (128 bytes, the swizzle span) x 128 rows; 128-byte swizzle;
-// out-of-range rows read as zero.
+// out-of-range rows, and columns past `cols` (a head dim below the kernel's
+// 64 / 128), read as zero.
 cudaError_t encode(TmaDesc* out, const FaParams& p, const void* base, int cols, int rows, int heads,
                    int64_t s_stride, int64_t n_stride, int64_t b_stride) {
     EncodeTiledFn fn = encode_fn();
@@ -1101,7 +1139,7 @@ cudaError_t encode(TmaDesc* out, const FaParams& p, const void* base, int cols, 
 cudaError_t make_sm100_tmaps(const FaParams& p, TmaSet* maps) {
     cudaError_t e = encode(&maps->q, p, p.q, p.D, p.Tq, p.Nq, p.q_s, p.q_n, p.q_b);
     if (e == cudaSuccess) e = encode(&maps->k, p, p.k, p.D, p.Tkv, p.Nkv, p.k_s, p.k_n, p.k_b);
-    if (e == cudaSuccess) e = encode(&maps->v, p, p.v, p.D, p.Tkv, p.Nkv, p.v_s, p.v_n, p.v_b);
+    if (e == cudaSuccess) e = encode(&maps->v, p, p.v, p.Dv, p.Tkv, p.Nkv, p.v_s, p.v_n, p.v_b);
     if (e != cudaSuccess) return e;
     if (p.Dr) {
         e = encode(&maps->qr, p, p.qr, p.Dr, p.Tq, p.Nq, p.qr_s, p.qr_n, p.qr_b);
@@ -1129,7 +1167,7 @@ uint64_t plan_sm100_schedule(FaParams& p, int num_sms, bool uniform, int item_kv
     p.n_whole = p.n_items - tail;
     p.n_pieces = pieces;
     p.n_tickets = p.n_whole + tail * pieces;
-    return static_cast<uint64_t>(tail) * pieces * kQBlock * (p.D + 4) * sizeof(float);
+    return static_cast<uint64_t>(tail) * pieces * kQBlock * part_row_words(p.D > 64 ? 128 : 64) * sizeof(float);
 }
 
 cudaError_t launch_sm100(const FaParams& p, const TmaSet& maps, int num_sms, cudaStream_t stream) {

@@ -178,7 +178,7 @@ extern "C" fa_status fa_fwd_varlen_static(
     auto tma_dim_ok = [](int64_t stride, int64_t size) {
         return size == 1 || (stride > 0 && (stride * 2) % 16 == 0 && stride * 2 < (int64_t(1) << 40));
     };
-    const bool sm100 = (dt == FA_F16 || dt == FA_BF16) && D == Dv && (D == 64 || D == 128) && aligned16(p.q) &&
+    const bool sm100 = (dt == FA_F16 || dt == FA_BF16) && D <= 128 && D % 8 == 0 && Dv % 8 == 0 && aligned16(p.q) &&
                        aligned16(p.k) && aligned16(p.v) && tma_dim_ok(qst, Tq) && tma_dim_ok(qsn, Nq) &&
                        tma_dim_ok(kst, Tk) && tma_dim_ok(ksn, Nk) && tma_dim_ok(vst, Tk) && tma_dim_ok(vsn, Nk);
 

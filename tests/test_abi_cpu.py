@@ -303,9 +303,22 @@ def test_head_dim_limits():
     q, k, _ = qkv((1, 2, 16, 64))
     v = torch.zeros(1, 2, 16, 96, dtype=torch.float16)  # value head dim above key's
     assert plan(q, k, v)[0] == fa.FA_ERR_INNER_NULLPTR
-    v = torch.zeros(1, 2, 16, 32, dtype=torch.float16)  # below is allowed (CUDA-core kernel)
+    v = torch.zeros(1, 2, 16, 32, dtype=torch.float16)  # below is allowed
     st, _, text = plan(q, k, v)
-    assert st == 0 and "simt" in text
+    assert st == 0 and "sm100_tcgen05" in text and "Dv=32" in text
+
+
+@pytest.mark.parametrize("d,dv,kernel", [(96, 96, "sm100_tcgen05"), (128, 64, "sm100_tcgen05"),
+                                         (32, 32, "sm100_tcgen05"), (80, 48, "sm100_tcgen05"),
+                                         (100, 100, "simt"), (64, 36, "simt"), (160, 160, "simt"),
+                                         (256, 256, "simt")])
+def test_plan_head_dims_route(d, dv, kernel):
+    # half types with D <= 128 and D, Dv multiples of 8 run zero-padded on the
+    # tensor cores; the rest on the CUDA-core kernel
+    q, k, _ = qkv((1, 2, 300, d))
+    v = torch.zeros(1, 2, 300, dv, dtype=torch.float16)
+    st, _, text = plan(q, k, v)
+    assert st == 0 and kernel in text
 
 
 def test_batch_and_seq_mismatch():

@@ -225,15 +225,52 @@ def test_fp32_features(layout):
     compare_full(w)
 
 
-@pytest.mark.parametrize("d", [32, 96, 256])
-def test_half_types_other_head_dims(d):
+@pytest.mark.parametrize("d,kernel", [(32, "sm100_tcgen05"), (96, "sm100_tcgen05"), (100, "simt"),
+                                      (256, "simt")])
+def test_half_types_other_head_dims(d, kernel):
     w = W("BNSD", "bf16", (1, 2, 150, d), 2, 1900 + d, next_tokens=0)
-    assert "simt" in plan_text(w)
+    assert kernel in plan_text(w)
     compare_full(w)
 
 
 def test_value_head_dim_smaller():
     w = W("BNSD", "f16", (1, 2, 100, 128), 2, 2000, vshape=(1, 2, 100, 64))
+    assert "sm100_tcgen05" in plan_text(w)
+    compare_full(w)
+
+
+# Head dims below the kernel's 64 / 128 columns (zero-padded by the loads):
+# dense with a split last wave (the merge kernel writes Dv columns), varlen
+# causal with a sink, BSH band with GQA, a value head dim that is not a
+# multiple of 32, and rope on top of D = 96.
+@pytest.mark.parametrize("dtype,d,dv", [("f16", 96, 96), ("bf16", 128, 64), ("bf16", 80, 48), ("f16", 48, 40),
+                                        ("bf16", 120, 88)])
+def test_padded_head_dims_split_dense(dtype, d, dv):
+    n = 19  # 152 items of 256 rows: on 148 SMs the last wave is split
+    w = W("BNSD", dtype, (1, n, 2048, d), n, 4000 + d + dv, vshape=(1, n, 2048, dv))
+    text = plan_text(w)
+    assert "sm100_tcgen05" in text
+    if _sms() == 148:
+        assert _split_of(w)[0] > 0
+    compare_full(w)
+
+
+@pytest.mark.parametrize("d,dv", [(96, 96), (128, 72), (40, 40)])
+def test_padded_head_dims_varlen_causal_sink(d, dv):
+    lens = [300, 0, 513, 129, 1]
+    t = sum(lens)
+    w = W("TND", "bf16", (t, 4, d), 4, 4100 + d, kshape=(t, 2, d), vshape=(t, 2, dv),
+          actual_seq_q=cumulative(lens, False), actual_seq_kv=cumulative(lens, False), next_tokens=0,
+          sink=normal((4,), "f32", 4150))
+    assert "sm100_tcgen05" in plan_text(w)
+    compare_full(w)
+
+
+def test_padded_head_dims_bsh_band_alibi():
+    w = W("BSH", "f16", (2, 300, 4 * 96), 4, 4200, kshape=(2, 300, 2 * 96), vshape=(2, 300, 2 * 56),
+          pre_tokens=90, next_tokens=30)
+    w.pse, w.pse_type = alibi_slopes(4), 2
+    assert "sm100_tcgen05" in plan_text(w)
     compare_full(w)
 
 
@@ -488,7 +525,7 @@ def test_rope_worked_example():
     check_stats(f64(ssum), np.full((t, 1, 8), t + np.exp(3.0 - m)), "softmaxSum")
 
 
-@pytest.mark.parametrize("case", ["tnd_gqa_causal_sink", "bnsd_d64", "bsh_band"])
+@pytest.mark.parametrize("case", ["tnd_gqa_causal_sink", "bnsd_d64", "bsh_band", "tnd_d96"])
 def test_rope_tcgen05(case):
     if case == "tnd_gqa_causal_sink":
         lens = [300, 0, 513, 129]
@@ -498,9 +535,15 @@ def test_rope_tcgen05(case):
                                next_tokens=0, sink=normal((4,), "f32", 3720))
     elif case == "bnsd_d64":
         w, qr, kr = _rope_case("BNSD", (2, 3, 300, 64), (2, 3, 333, 64), (2, 3, 300, 64), (2, 3, 333, 64), 3, 3730)
-    else:
+    elif case == "bsh_band":
         w, qr, kr = _rope_case("BSH", (2, 260, 2 * 128), (2, 260, 2 * 128), (2, 260, 2 * 64), (2, 260, 2 * 64), 2,
                                3740, pre_tokens=100, next_tokens=20)
+    else:
+        lens = [200, 333]
+        t = sum(lens)
+        w, qr, kr = _rope_case("TND", (t, 2, 96), (t, 2, 96), (t, 2, 64), (t, 2, 64), 2, 3760,
+                               actual_seq_q=cumulative(lens, False), actual_seq_kv=cumulative(lens, False),
+                               next_tokens=0)
     _rope_compare(w, qr, kr, "sm100_tcgen05")
 
 
