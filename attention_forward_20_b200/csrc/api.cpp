@@ -403,7 +403,7 @@ extern "C" fa_status fa_fwd_get_workspace_size_v5(
                 p.pse_n % 8 == 0 && p.pse_i % 8 == 0;
 
     // ---- kernel choice -------------------------------------------------------
-    // tcgen05 needs fp16/bf16, D <= 128, and TMA-legal operands:
+    // tcgen05 needs fp16/bf16, D <= 256, and TMA-legal operands:
     // 16-byte aligned bases and, for every dimension longer than 1, a positive
     // byte stride that is a multiple of 16 and below 2^40.
     auto tma_dim_ok = [](int64_t stride, int64_t size) {
@@ -421,9 +421,9 @@ extern "C" fa_status fa_fwd_get_workspace_size_v5(
         tma_ok = tma_ok && p.Dr == 64 && aligned16(p.qr) && aligned16(p.kr) && tma_dim_ok(p.qr_s, qv.S) &&
                  tma_dim_ok(p.qr_n, qv.N) && tma_dim_ok(p.qr_b, qB) && tma_dim_ok(p.kr_s, kv.S) &&
                  tma_dim_ok(p.kr_n, kv.N) && tma_dim_ok(p.kr_b, qB);
-    // head dims: D <= 128 and Dv <= D, multiples of 8 (whole 16-byte pieces of
-    // a row), run zero-padded to 64 or 128 columns
-    const bool dims_ok = qv.D <= 128 && qv.D % 8 == 0 && vv.D % 8 == 0;
+    // head dims: D <= 256 and Dv <= D, multiples of 8 (whole 16-byte pieces of
+    // a row), run zero-padded to 64, 128 or 256 columns (rope: D <= 128)
+    const bool dims_ok = qv.D <= 256 && qv.D % 8 == 0 && vv.D % 8 == 0 && (!rope || qv.D <= 128);
     const bool sm100 = (dt == FA_F16 || dt == FA_BF16) && dims_ok && tma_ok;
     ex->kind = sm100 ? fa::KERNEL_SM100 : fa::KERNEL_SIMT;
 

@@ -87,8 +87,8 @@ struct Cfg {
     static constexpr int kStages = (D == 128) ? (kRope ? 3 : 4) : 8;  // K/V ring slots
     static constexpr int kSmemBytes = 2 * kQTileBytes + kStages * kTileBytes + kRopeSlots * kChunkBytes + 1024;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kOCol = 256;
 };
+constexpr uint32_t kOCol = 256;  // TMEM column of O (S and P use 0..255)
 static_assert(Cfg<128, true>::kSmemBytes + 1024 <= 227 * 1024, "rope tiles exceed shared memory");
 static_assert(Cfg<64, true>::kSmemBytes + 1024 <= 227 * 1024, "rope tiles exceed shared memory");
 
@@ -96,6 +96,7 @@ struct Barriers {
     uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2];
     uint64_t kv_full[8], kv_empty[8];
     uint64_t kr_empty[2];  // keyRope slots (the K load's kv_full also covers its keyRope chunk)
+    uint64_t pv_done;      // wide kernel: one completion per key block's P·V
     uint64_t sched_full[kSched], sched_empty[kSched];
     uint64_t drain;
     uint64_t never;  // failure injection: initialised, never arrived on
@@ -418,7 +419,7 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* s
     };
     auto issue_pv = [&](int t, int slot, bool accumulate) {
         const uint64_t vd = sdesc_sw128(smem_u32(sKV + slot * C::kTileBytes), 1024, C::kChunkBytes);
-        if (elect_one()) mma_ts_k128(tmem + C::kOCol + t * D, tmem + t * kTileN, vd, idesc_pv, accumulate ? 1u : 0u);
+        if (elect_one()) mma_ts_k128(tmem + kOCol + t * D, tmem + t * kTileN, vd, idesc_pv, accumulate ? 1u : 0u);
         __syncwarp();
     };
 
@@ -478,6 +479,189 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* s
             if (tr[t].active()) ++q_use[t];
     }
     // Drain: every MMA this warp issued completes before TMEM is freed.
+    commit(&bars.drain);
+    warp_wait(&bars.drain, 0, abort, kSiteDrain);
+}
+
+// ---------------------------------------------------------------------------
+// Wide kernel (head dims 129..256, zero-padded to 256): one query tile at a
+// time.  TMEM: S in two buffers (columns 0 and 128) that alternate from key
+// block to key block, O at 256..511.  Shared memory: the Q tile (64 KB) and a
+// ring of kWideSlots half-tiles (128 rows x 128 columns, 32 KB): K of a block
+// is two halves, V one or two (by Dv).  Ring order per tile: K_lo, K_lo+1,
+// then V_j, K_j+2 for j = lo .. hi, which is the order the MMA warp uses them.
+// ---------------------------------------------------------------------------
+constexpr int kWideSlots = 5;
+constexpr int kWideThreads = 192;  // softmax warps 0-3, TMA warp 4, MMA warp 5
+constexpr int kWideLoadWarp = 4;
+constexpr int kWideMmaWarp = 5;
+constexpr int kHalfBytes = kTileM * 128 * 2;  // 128 rows x 128 columns
+constexpr int kWideQBytes = kTileM * 256 * 2;
+constexpr int kWideSmemBytes = kWideQBytes + kWideSlots * kHalfBytes + 1024;
+static_assert(kWideSmemBytes + 1024 <= 227 * 1024, "wide kernel tiles exceed shared memory");
+
+__device__ void run_producer_wide(const FaParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
+                                  const CUtensorMap* tv, uint8_t* sQ, uint8_t* sKV, Barriers& bars,
+                                  TicketSlots& slots, volatile int* abort) {
+    constexpr int kChunkBytes = kTileM * 128;
+    uint32_t fill = 0, q_fill = 0, k_sched = 0;
+    bool ok = true;
+    const int v_halves = (p.Dv + 127) / 128;
+
+    while (ok) {
+        Item tit;
+        const int ticket = take_ticket_global(p, bars, slots, k_sched, tit, abort);
+        if (ticket == kTicketAbort) { ok = false; break; }
+        if (ticket == kTicketEnd) break;
+        const Work wk = work_of(p, ticket, tit);
+        const Item it = wk.it;
+        auto load_chunk = [&](const CUtensorMap* tm, uint8_t* dst, uint64_t* bar, int c, int row, int head) {
+            if (p.varlen)
+                tma_load_3d(dst, tm, bar, c * 64, (int)(it.kv_off + row), head);
+            else
+                tma_load_4d(dst, tm, bar, c * 64, row, head, it.b);
+        };
+        // one half (columns 128h .. 128h+127) of key block jb of K or V
+        auto load_half = [&](const CUtensorMap* tm, int jb, int h) -> bool {
+            const int slot = fill % kWideSlots;
+            if (!warp_wait(&bars.kv_empty[slot], ((fill / kWideSlots) & 1) ^ 1, abort, kSiteKvEmpty)) return false;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&bars.kv_full[slot], kHalfBytes);
+                uint8_t* dst = sKV + slot * kHalfBytes;
+                load_chunk(tm, dst, &bars.kv_full[slot], 2 * h, jb * kTileN, it.nk);
+                load_chunk(tm, dst + kChunkBytes, &bars.kv_full[slot], 2 * h + 1, jb * kTileN, it.nk);
+            }
+            __syncwarp();
+            ++fill;
+            return true;
+        };
+        auto load_k = [&](int jb) { return load_half(tk, jb, 0) && load_half(tk, jb, 1); };
+        auto load_v = [&](int jb) {
+            for (int h = 0; h < v_halves; ++h)
+                if (!load_half(tv, jb, h)) return false;
+            return true;
+        };
+        for (int tt = 0; tt < 2 && ok; ++tt) {
+            const TileRange tr = tt ? wk.tr[1] : wk.tr[0];
+            if (!tr.active()) continue;
+            if (!warp_wait(&bars.q_empty[0], (q_fill & 1) ^ 1, abort, kSiteQEmpty)) { ok = false; break; }
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&bars.q_full[0], kWideQBytes);
+                const int row = it.qb * kQBlock + tt * kTileM;
+                for (int c = 0; c < 4; ++c) {
+                    if (p.varlen)
+                        tma_load_3d(sQ + c * kChunkBytes, tq, &bars.q_full[0], c * 64, (int)(it.q_off + row), it.n);
+                    else
+                        tma_load_4d(sQ + c * kChunkBytes, tq, &bars.q_full[0], c * 64, row, it.n, it.b);
+                }
+            }
+            __syncwarp();
+            ++q_fill;
+            if (!load_k(tr.lo) || (tr.lo + 1 <= tr.hi && !load_k(tr.lo + 1))) { ok = false; break; }
+            for (int jb = tr.lo; jb <= tr.hi; ++jb) {
+                if (!load_v(jb) || (jb + 2 <= tr.hi && !load_k(jb + 2))) { ok = false; break; }
+            }
+        }
+    }
+    // Drain: the latest fill of every slot and of Q has landed.
+    for (int sl = 0; sl < kWideSlots; ++sl) {
+        if ((uint32_t)sl < fill) {
+            const uint32_t last = fill - 1 - ((fill - 1 - sl) % kWideSlots);
+            mbar_wait(&bars.kv_full[sl], (last / kWideSlots) & 1, abort, kSiteDrain);
+        }
+    }
+    if (q_fill) mbar_wait(&bars.q_full[0], (q_fill - 1) & 1, abort, kSiteDrain);
+}
+
+template <typename T>
+__device__ void run_mma_wide(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barriers& bars, const TicketSlots& slots,
+                             uint32_t tmem, volatile int* abort) {
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    constexpr int kChunkBytes = kTileM * 128;
+    const uint32_t idesc_qk = idesc_f16(kBf16, kTileM, kTileN, false, false, p.neg_scale != 0);
+    constexpr uint32_t idesc_pv = idesc_f16(kBf16, kTileM, 128, false, true, false);
+    const int v_halves = (p.Dv + 127) / 128;
+    uint32_t use = 0, q_use = 0, p_cnt0 = 0, p_cnt1 = 0, k_sched = 0, g = 0;
+    bool ok = true;
+    if (p.debug_stall && !warp_wait(&bars.never, 0, abort, kSiteInjected)) ok = false;
+
+    auto wait_half = [&](int* slot) -> bool {
+        *slot = use % kWideSlots;
+        const bool r = warp_wait(&bars.kv_full[*slot], (use / kWideSlots) & 1, abort, kSiteKvFull);
+        ++use;
+        return r;
+    };
+    auto commit = [&](uint64_t* bar) {
+        if (elect_one()) tc_commit(bar);
+        __syncwarp();
+    };
+    // S_b = Q · K^T over 256 columns: K-steps 0..7 against K's first half,
+    // 8..15 (Q chunks 2, 3) against its second half.
+    auto qk = [&](uint32_t b) -> bool {
+        int k0, k1;
+        if (!wait_half(&k0) || !wait_half(&k1)) return false;
+        tc_fence_after();
+        const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 1024, 16);
+        const uint64_t qd2 = sdesc_sw128(smem_u32(sQ + 2 * kChunkBytes), 1024, 16);
+        const uint64_t kd0 = sdesc_sw128(smem_u32(sKV + k0 * kHalfBytes), 1024, 16);
+        const uint64_t kd1 = sdesc_sw128(smem_u32(sKV + k1 * kHalfBytes), 1024, 16);
+        if (elect_one()) {
+            mma_ss_k128(tmem + b * kTileN, qd0, kd0, idesc_qk, 0u);
+            mma_ss_k128(tmem + b * kTileN, qd2, kd1, idesc_qk, 1u);
+        }
+        __syncwarp();
+        commit(&bars.s_full[b]);
+        commit(&bars.kv_empty[k0]);
+        commit(&bars.kv_empty[k1]);
+        return true;
+    };
+
+    while (ok) {
+        Item tit;
+        const int ticket = take_ticket_local(p, bars, slots, k_sched, tit, abort);
+        if (ticket == kTicketAbort) { ok = false; break; }
+        if (ticket == kTicketEnd) break;
+        const Work wk = work_of(p, ticket, tit);
+        for (int tt = 0; tt < 2 && ok; ++tt) {
+            const TileRange tr = tt ? wk.tr[1] : wk.tr[0];
+            if (!tr.active()) continue;
+            if (!warp_wait(&bars.q_full[0], q_use & 1, abort, kSiteQFull)) { ok = false; break; }
+            ++q_use;
+            if (!qk(g & 1)) { ok = false; break; }
+            if (tr.lo == tr.hi) commit(&bars.q_empty[0]);
+            if (tr.lo + 1 <= tr.hi) {
+                if (!qk((g + 1) & 1)) { ok = false; break; }
+                if (tr.lo + 1 == tr.hi) commit(&bars.q_empty[0]);
+            }
+            for (int jb = tr.lo; jb <= tr.hi; ++jb, ++g) {
+                const uint32_t b = g & 1;
+                int v0 = 0, v1 = 0;
+                if (!wait_half(&v0) || (v_halves > 1 && !wait_half(&v1))) { ok = false; break; }
+                const uint32_t pc = b ? p_cnt1 : p_cnt0;
+                if (!warp_wait(&bars.p_full[b], pc & 1, abort, kSitePFull)) { ok = false; break; }
+                if (b) ++p_cnt1; else ++p_cnt0;
+                tc_fence_after();
+                const uint32_t acc = jb != tr.lo ? 1u : 0u;
+                const uint64_t vd0 = sdesc_sw128(smem_u32(sKV + v0 * kHalfBytes), 1024, kChunkBytes);
+                if (elect_one()) mma_ts_k128(tmem + 256, tmem + b * kTileN, vd0, idesc_pv, acc);
+                __syncwarp();
+                if (v_halves > 1) {
+                    const uint64_t vd1 = sdesc_sw128(smem_u32(sKV + v1 * kHalfBytes), 1024, kChunkBytes);
+                    if (elect_one()) mma_ts_k128(tmem + 384, tmem + b * kTileN, vd1, idesc_pv, acc);
+                    __syncwarp();
+                }
+                commit(&bars.pv_done);
+                commit(&bars.kv_empty[v0]);
+                if (v_halves > 1) commit(&bars.kv_empty[v1]);
+                if (jb == tr.hi) commit(&bars.o_full[0]);
+                if (jb + 2 <= tr.hi) {
+                    // into the buffer whose P this block's P·V reads: issued after it
+                    if (!qk(b)) { ok = false; break; }
+                    if (jb + 2 == tr.hi) commit(&bars.q_empty[0]);
+                }
+            }
+        }
+    }
     commit(&bars.drain);
     warp_wait(&bars.drain, 0, abort, kSiteDrain);
 }
@@ -638,17 +822,20 @@ __device__ __forceinline__ void store_stats(const FaParams& p, const Item& it, i
 
 // kBias: 0 no bias, 1 dense bias tensor, 2 ALiBi slopes (one variant each, so
 // that each kernel carries only its own bias code).
-template <typename T, int D, int kBias>
+// Two-tile kernels: warpgroup t owns query tile t of every item, S_t at
+// columns 128t, O_t at kOCol + tD.  kWide (head dims above 128): the one
+// softmax warpgroup takes both tiles of an item in turn; S alternates between
+// the buffers at columns 0 and 128 from one key block to the next, O is at
+// kOCol, and a rescale of O first waits for the previous block's P·V (pv_done).
+template <typename T, int D, int kBias, bool kWide = false>
 __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots& slots, uint32_t tmem,
                             volatile int* abort, int t) {
-    using C = Cfg<D>;
     const int quad = (threadIdx.x >> 5) & 3;
     const int row = quad * 32 + (threadIdx.x & 31);
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off + t * kTileN;
-    const uint32_t tO = tmem + lane_off + C::kOCol + t * D;
+    const uint32_t tO = tmem + lane_off + kOCol + t * D;
     const float sl2 = p.scale_log2;
-    uint32_t s_cnt = 0, o_cnt = 0, k_sched = 0;
+    uint32_t s_cnt0 = 0, s_cnt1 = 0, o_cnt = 0, k_sched = 0, g_blk = 0;
     bool ok = true;
 
     while (ok) {
@@ -658,9 +845,10 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
         if (ticket == kTicketEnd) break;
         const Work wk = work_of(p, ticket, tit);
         const Item it = wk.it;
-        const TileRange tr = t ? wk.tr[1] : wk.tr[0];  // a select: no indexing of wk by a runtime value
+      for (int tt = kWide ? 0 : t; tt <= (kWide ? 1 : t); ++tt) {
+        const TileRange tr = tt ? wk.tr[1] : wk.tr[0];  // a select: no indexing of wk by a runtime value
         if (!tr.valid) continue;
-        const int r0 = it.qb * kQBlock + t * kTileM;
+        const int r0 = it.qb * kQBlock + tt * kTileM;
         const int i = r0 + row;
         const bool row_ok = i < it.q_len;
 
@@ -689,8 +877,11 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                     if (jn + 64 < pse_cols) prefetch_l2(pse_row + jn + 64);
                 }
             }
-            if (!warp_wait(&bars.s_full[t], s_cnt & 1, abort, kSiteSFull)) { ok = false; break; }
-            ++s_cnt;
+            const uint32_t sb = kWide ? (g_blk & 1u) : static_cast<uint32_t>(t);
+            const uint32_t sc = (kWide && sb) ? s_cnt1 : s_cnt0;
+            if (!warp_wait(&bars.s_full[sb], sc & 1, abort, kSiteSFull)) { ok = false; break; }
+            if (kWide && sb) ++s_cnt1; else ++s_cnt0;
+            const uint32_t tS = tmem + lane_off + sb * kTileN;
             tc_fence_after();
             float s[128];
             {
@@ -814,8 +1005,11 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
             l += (l0 + l1) + (l2 + l3);
             tmem_st_x64(tS, pk);
             if (jb > tr.lo && __any_sync(0xffffffffu, need)) {
-                // Rescale O_t by alpha before this block's P·V is issued.  O_t is
-                // stable: the commit behind this block's S_t covered the last P·V.
+                // Rescale O_t by alpha before this block's P·V is issued.  Two
+                // tiles: O_t is stable, the commit behind this block's S_t covered
+                // the last P·V.  Wide: wait for the previous block's P·V.
+                if (kWide && !warp_wait(&bars.pv_done, (g_blk - 1) & 1, abort, kSiteOFull)) { ok = false; break; }
+                if (kWide) tc_fence_after();
 #pragma unroll
                 for (int cc = 0; cc < D; cc += 32) {
                     if (cc >= p.Dv) break;
@@ -828,7 +1022,8 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars.p_full[t]);
+            mbar_arrive(&bars.p_full[sb]);
+            if (kWide) ++g_blk;
         }
         if (!ok) break;
 
@@ -842,7 +1037,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
         if (wk.piece >= 0) {
             // A piece of a split item: keep O_t (relative to m_used) and the
             // row's m_run, m_used, l for the merge.
-            float* prow = p.part + ((static_cast<size_t>(wk.tail) * p.n_pieces + wk.piece) * kQBlock + t * kTileM + row) *
+            float* prow = p.part + ((static_cast<size_t>(wk.tail) * p.n_pieces + wk.piece) * kQBlock + tt * kTileM + row) *
                                        static_cast<size_t>(D + 4);
 #pragma unroll 1
             for (int cc = 0; cc < D; cc += 32) {
@@ -880,6 +1075,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                 store_out8s<T>(p, orow, cc, (p.Dv - cc) / 8, o, f.o_scale);
         }
         if (row_ok) store_stats(p, it, i, f);
+      }
     }
 }
 
@@ -1028,6 +1224,88 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicCAS(&g_fa_error, 0ull, (static_cast<unsigned long long>(abort_flag) << 32) | (blockIdx.x + 1u));
 }
 
+// Wide kernel: head dims 129..256 (see run_producer_wide).
+template <typename T, int kBias>
+__global__ void __launch_bounds__(kWideThreads, 1)
+    fa_fwd_sm100_wide_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                             const __grid_constant__ CUtensorMap tmap_v, const FaParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = smem;
+    uint8_t* sKV = smem + kWideQBytes;
+    __shared__ Barriers bars;
+    __shared__ TicketSlots slots;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&bars.q_full[0], 1);
+        mbar_init(&bars.q_empty[0], 1);
+        mbar_init(&bars.o_full[0], 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars.s_full[b], 1);
+            mbar_init(&bars.p_full[b], kTileM);
+        }
+        for (int sl = 0; sl < kWideSlots; ++sl) {
+            mbar_init(&bars.kv_full[sl], 1);
+            mbar_init(&bars.kv_empty[sl], 1);
+        }
+        for (int k = 0; k < kSched; ++k) {
+            mbar_init(&bars.sched_full[k], 1);
+            mbar_init(&bars.sched_empty[k], 5);  // the MMA warp and the four softmax warps
+        }
+        mbar_init(&bars.pv_done, 1);
+        mbar_init(&bars.drain, 1);
+        mbar_init(&bars.never, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kWideLoadWarp && lane == 0) {
+        prefetch_tmap(&tmap_q);
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_v);
+    }
+    if (warp == kWideMmaWarp) {
+        tmem_alloc(&tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+
+    if (warp < 4)
+        run_softmax<T, 256, kBias, true>(p, bars, slots, tmem, &abort_flag, 0);
+    else if (warp == kWideLoadWarp)
+        run_producer_wide(p, &tmap_q, &tmap_k, &tmap_v, sQ, sKV, bars, slots, &abort_flag);
+    else if (warp == kWideMmaWarp)
+        run_mma_wide<T>(p, sQ, sKV, bars, slots, tmem, &abort_flag);
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWideMmaWarp) tmem_dealloc(tmem, 512);
+    if (threadIdx.x == 0 && abort_flag != 0)
+        atomicCAS(&g_fa_error, 0ull, (static_cast<unsigned long long>(abort_flag) << 32) | (blockIdx.x + 1u));
+}
+
+template <typename T, int kBias>
+cudaError_t launch_wide(const FaParams& p, const TmaSet& maps, cudaStream_t stream) {
+    auto kern = fa_fwd_sm100_wide_kernel<T, kBias>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kWideSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (p.grid <= 0) return cudaSuccess;
+    auto map = [](const TmaDesc& d) -> const CUtensorMap& { return *reinterpret_cast<const CUtensorMap*>(&d); };
+    kern<<<p.grid, kWideThreads, kWideSmemBytes, stream>>>(map(maps.q), map(maps.k), map(maps.v), p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.n_pieces == 0) return e;
+    const int n_split = (p.n_tickets - p.n_whole) / p.n_pieces;
+    const int merge_threads = n_split * kQBlock * (256 / 8);
+    fa_merge_kernel<T, 256><<<(merge_threads + kMergeThreads - 1) / kMergeThreads, kMergeThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
 template <typename T, int D, int kBias, bool kRope = false>
 cudaError_t launch_t(const FaParams& p, const TmaSet& maps, int num_sms, cudaStream_t stream) {
     using C = Cfg<D, kRope>;
@@ -1060,7 +1338,13 @@ cudaError_t launch_d(const FaParams& p, const TmaSet& maps, int num_sms, cudaStr
     // pse_type is 0 whenever realShift is absent; rope (bf16 only, no
     // realShift) has kernels of its own
     // head dims up to 64 run on the 64-column kernels, up to 128 on the
-    // 128-column ones (columns past D and Dv load as zero)
+    // 128-column ones, up to 256 on the wide kernel (columns past D and Dv
+    // load as zero)
+    if (p.D > 128) {
+        if (p.pse_type == 2) return launch_wide<T, 2>(p, maps, stream);
+        if (p.pse_type == 1) return launch_wide<T, 1>(p, maps, stream);
+        return launch_wide<T, 0>(p, maps, stream);
+    }
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         if (p.Dr) {
             if (p.D > 64) return launch_t<T, 128, 0, true>(p, maps, num_sms, stream);
@@ -1167,7 +1451,8 @@ uint64_t plan_sm100_schedule(FaParams& p, int num_sms, bool uniform, int item_kv
     p.n_whole = p.n_items - tail;
     p.n_pieces = pieces;
     p.n_tickets = p.n_whole + tail * pieces;
-    return static_cast<uint64_t>(tail) * pieces * kQBlock * part_row_words(p.D > 64 ? 128 : 64) * sizeof(float);
+    const int d_pad = p.D > 128 ? 256 : (p.D > 64 ? 128 : 64);
+    return static_cast<uint64_t>(tail) * pieces * kQBlock * part_row_words(d_pad) * sizeof(float);
 }
 
 cudaError_t launch_sm100(const FaParams& p, const TmaSet& maps, int num_sms, cudaStream_t stream) {

@@ -310,11 +310,16 @@ def test_head_dim_limits():
 
 @pytest.mark.parametrize("d,dv,kernel", [(96, 96, "sm100_tcgen05"), (128, 64, "sm100_tcgen05"),
                                          (32, 32, "sm100_tcgen05"), (80, 48, "sm100_tcgen05"),
-                                         (100, 100, "simt"), (64, 36, "simt"), (160, 160, "simt"),
-                                         (256, 256, "simt")])
+                                         (100, 100, "simt"), (64, 36, "simt"), (160, 160, "sm100_tcgen05"),
+                                         (256, 256, "sm100_tcgen05"), (192, 128, "sm100_tcgen05"),
+                                         (264, 264, "simt")])
 def test_plan_head_dims_route(d, dv, kernel):
-    # half types with D <= 128 and D, Dv multiples of 8 run zero-padded on the
-    # tensor cores; the rest on the CUDA-core kernel
+    # half types with D <= 256 and D, Dv multiples of 8 run zero-padded on the
+    # tensor cores; the rest on the CUDA-core kernel (up to 256; 264 is rejected)
+    if d > 256:
+        q, k, v = qkv((1, 2, 300, d))
+        assert plan(q, k, v)[0] == fa.FA_ERR_INNER_NULLPTR
+        return
     q, k, _ = qkv((1, 2, 300, d))
     v = torch.zeros(1, 2, 300, dv, dtype=torch.float16)
     st, _, text = plan(q, k, v)

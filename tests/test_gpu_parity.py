@@ -226,7 +226,7 @@ def test_fp32_features(layout):
 
 
 @pytest.mark.parametrize("d,kernel", [(32, "sm100_tcgen05"), (96, "sm100_tcgen05"), (100, "simt"),
-                                      (256, "simt")])
+                                      (256, "sm100_tcgen05"), (204, "simt")])
 def test_half_types_other_head_dims(d, kernel):
     w = W("BNSD", "bf16", (1, 2, 150, d), 2, 1900 + d, next_tokens=0)
     assert kernel in plan_text(w)
@@ -263,6 +263,46 @@ def test_padded_head_dims_varlen_causal_sink(d, dv):
           actual_seq_q=cumulative(lens, False), actual_seq_kv=cumulative(lens, False), next_tokens=0,
           sink=normal((4,), "f32", 4150))
     assert "sm100_tcgen05" in plan_text(w)
+    compare_full(w)
+
+
+# Head dims 129..256: the wide kernel (one query tile at a time, S
+# double-buffered, K/V in 128-column halves).
+@pytest.mark.parametrize("dtype,d,dv", [("bf16", 256, 256), ("f16", 192, 128), ("bf16", 160, 96)])
+def test_wide_head_dims_split_dense(dtype, d, dv):
+    n = 19  # 152 items: the last wave is split and merged
+    w = W("BNSD", dtype, (1, n, 2048, d), n, 4300 + d + dv, vshape=(1, n, 2048, dv))
+    assert "sm100_tcgen05" in plan_text(w)
+    if _sms() == 148:
+        assert _split_of(w)[0] > 0
+    compare_full(w)
+
+
+@pytest.mark.parametrize("d,dv", [(256, 256), (224, 136)])
+def test_wide_head_dims_varlen_causal_sink_gqa(d, dv):
+    lens = [300, 0, 513, 129, 1, 640]
+    t = sum(lens)
+    w = W("TND", "bf16", (t, 4, d), 4, 4400 + d, kshape=(t, 2, d), vshape=(t, 2, dv),
+          actual_seq_q=cumulative(lens, False), actual_seq_kv=cumulative(lens, False), next_tokens=0,
+          sink=normal((4,), "f32", 4450))
+    assert "sm100_tcgen05" in plan_text(w)
+    compare_full(w)
+
+
+def test_wide_head_dims_band_alibi_and_dense_bias_and_mask():
+    w = W("BSH", "f16", (2, 420, 2 * 256), 2, 4500, pre_tokens=150, next_tokens=40)
+    w.pse, w.pse_type = alibi_slopes(2), 2
+    compare_full(w)
+    w2 = W("BNSD", "bf16", (1, 2, 333, 256), 2, 4510, kshape=(1, 2, 400, 256), sink=normal((2,), "f32", 4520))
+    w2.pse, w2.pse_type = normal((1, 2, 333, 400), "bf16", 4530), 1
+    w2.atten_mask = (torch.rand(333, 400, generator=torch.Generator().manual_seed(4540)) < 0.2).to(torch.uint8)
+    compare_full(w2)
+
+
+def test_wide_head_dims_negative_scale_and_single_rows():
+    w = W("BNSD", "f16", (1, 2, 1, 256), 2, 4600, kshape=(1, 2, 5, 256), scale=-0.05)
+    compare_full(w)
+    w = W("BNSD", "bf16", (2, 2, 129, 256), 2, 4610, kshape=(2, 2, 1, 256))
     compare_full(w)
 
 
