@@ -107,13 +107,9 @@ def status_string(status):
     return load().fa_status_string(int(status)).decode()
 
 
+_Dims = ctypes.c_int64 * 8
+
+
 def make_tensor(data_ptr, dtype_code, shape, strides):
     """fa_tensor from a raw device address, dtype code, shape and element strides."""
-    t = FaTensor()
-    t.data = ctypes.c_void_p(int(data_ptr))
-    t.dtype = int(dtype_code)
-    t.ndim = len(shape)
-    for i, (s, st) in enumerate(zip(shape, strides)):
-        t.shape[i] = int(s)
-        t.strides[i] = int(st)
-    return t
+    return FaTensor(int(data_ptr), int(dtype_code), len(shape), _Dims(*shape), _Dims(*strides))

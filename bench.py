@@ -472,36 +472,63 @@ def main():
     if status != 0:
         raise SystemExit(f"kernel error word {word:#x}")
 
-    # end to end: pinned host inputs -> device, forward, result -> pinned host
+    # End to end through fa_fwd with host buffers: every step copies its inputs
+    # from pinned host memory and its results (output and statistics) back to
+    # pinned host memory.  Consecutive steps overlap on three streams (copy in,
+    # compute, copy out) with two sets of device buffers, as a serving loop
+    # would: step i+1's inputs travel while step i computes and step i-1's
+    # results return.
     host = [t.pin_memory() for t in (w.q, w.k, w.v) + (tuple(rope) if rope is not None else ())]
-    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    host_sm = torch.empty(smax.shape, dtype=smax.dtype).pin_memory()
-    host_ss = torch.empty(ssum.shape, dtype=ssum.dtype).pin_memory()
-    dev_in = [torch.empty_like(t, device=dev) for t in host]
-    dq, dk, dv = dev_in[:3]
-    kw_e2e = dict(kw, **({"query_rope": dev_in[3], "key_rope": dev_in[4]} if rope is not None else {}))
-    e2e_steps = max(3, min(args.steps, 20))
+    n_slots = 2
+    dev_in = [[torch.empty_like(t, device=dev) for t in host] for _ in range(n_slots)]
+    dev_res = [tuple(torch.empty_like(t) for t in (out, smax, ssum)) for _ in range(n_slots)]
+    host_res = [tuple(torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (out, smax, ssum))
+                for _ in range(n_slots)]
+    s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_ready = [torch.cuda.Event() for _ in range(n_slots)]
+    comp_done = [torch.cuda.Event() for _ in range(n_slots)]
+    out_done = [torch.cuda.Event() for _ in range(n_slots)]
+    used = [False] * n_slots
+    e2e_steps = max(4, min(args.steps, 20))
 
-    def e2e_step():
-        for d_, h_ in zip(dev_in, host):
-            d_.copy_(h_, non_blocking=True)
-        fa.fa_fwd(dq, dk, dv, out=out, softmax_max=smax, softmax_sum=ssum, **kw_e2e)
-        host_out.copy_(out, non_blocking=True)
-        host_sm.copy_(smax, non_blocking=True)
-        host_ss.copy_(ssum, non_blocking=True)
+    def e2e_step(i):
+        k_ = i % n_slots
+        if used[k_]:
+            s_in.wait_event(comp_done[k_])     # the forward that read these input buffers is done
+        with torch.cuda.stream(s_in):
+            for d_, h_ in zip(dev_in[k_], host):
+                d_.copy_(h_, non_blocking=True)
+        in_ready[k_].record(s_in)
+        s_comp.wait_event(in_ready[k_])
+        if used[k_]:
+            s_comp.wait_event(out_done[k_])    # these result buffers have been copied out
+        with torch.cuda.stream(s_comp):
+            kw_i = dict(kw, **({"query_rope": dev_in[k_][3], "key_rope": dev_in[k_][4]} if rope is not None else {}))
+            o_, m_, l_ = dev_res[k_]
+            fa.fa_fwd(dev_in[k_][0], dev_in[k_][1], dev_in[k_][2], out=o_, softmax_max=m_, softmax_sum=l_, **kw_i)
+        comp_done[k_].record(s_comp)
+        s_out.wait_event(comp_done[k_])
+        with torch.cuda.stream(s_out):
+            for h_, d_ in zip(host_res[k_], dev_res[k_]):
+                h_.copy_(d_, non_blocking=True)
+        out_done[k_].record(s_out)
+        used[k_] = True
 
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(s_out)                           # after the last step's results reached the host
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    # the last step's results equal the device-timed run's (same inputs, same call)
+    if args.kv_chunks == 1 and not torch.equal(host_res[(e2e_steps - 1) % n_slots][0], out.cpu()):
+        raise SystemExit("end-to-end result differs from the device-timed result")
     h2d = sum(t.numel() * t.element_size() for t in host)
-    d2h = sum(t.numel() * t.element_size() for t in (host_out, host_sm, host_ss))
+    d2h = sum(t.numel() * t.element_size() for t in host_res[0])
 
     kernel_ms, e2e_ms = max_over_ranks([kernel_ms, e2e_ms], dist, dev)
     if dist:
@@ -548,7 +575,8 @@ def main():
                                    f"{secs:.1f} s" + ("" if args.pse == "slopes" else
                                                       " (bias from the slopes, the same values in float64)")},
         "e2e": {"value": whole_job_tflops(flops_tiles, world, e2e_ms), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "pipeline": "copy in / compute / copy out on three streams, two buffer sets"},
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clocks.summary(),
     }
