@@ -486,3 +486,21 @@ def test_merge_validation():
     bad = torch.zeros(1, 2, 41, 64, dtype=torch.float16)
     assert _merge_status([bad], [st], [st], out, st, st) == _abi.FA_ERR_INNER_NULLPTR  # shape
     assert _merge_status([out], [torch.zeros(1, 2, 40, 4)], [st], out, st, st) == _abi.FA_ERR_INNER_NULLPTR
+
+
+def test_limits_rejected_one_past():
+    # S and T up to 1M, heads up to 256 (aclnnFlashAttentionVarLenScoreV5, 约束说明)
+    q = torch.zeros(1, 1, (1 << 20) + 1, 8, dtype=torch.float16)
+    assert plan(q, q, q)[0] == fa.FA_ERR_INNER_NULLPTR
+    q = torch.zeros(1, 1, 1 << 20, 8, dtype=torch.float16)
+    assert plan(q, q, q)[0] == 0
+    q = torch.zeros(1, 257, 4, 8, dtype=torch.float16)
+    assert plan(q, q, q)[0] == fa.FA_ERR_INNER_NULLPTR
+    # B up to 20000 sequences
+    t = torch.zeros(20001, 1, 8, dtype=torch.float16)
+    cum = list(range(1, 20002))
+    assert plan(t, t, t, input_layout="TND", head_num=1, actual_seq_qlen=cum,
+                actual_seq_kvlen=cum)[0] == fa.FA_ERR_INNER_NULLPTR
+    t = torch.zeros(20000, 1, 8, dtype=torch.float16)
+    cum = list(range(1, 20001))
+    assert plan(t, t, t, input_layout="TND", head_num=1, actual_seq_qlen=cum, actual_seq_kvlen=cum)[0] == 0

@@ -621,3 +621,44 @@ def test_full_size_varlen_with_rope_sampled():
     check_out(o, wo, "bf16", "sampled attentionOut rows")
     check_stats(m, wm, "sampled softmaxMax")
     check_stats(l, wl, "sampled softmaxSum")
+
+
+# ---------------------------------------------------------------------------
+# The operator's limits (aclnnFlashAttentionVarLenScoreV5, 约束说明: S and T up
+# to 1M, B up to 20000, N up to 256), sampled rows against the oracle
+# ---------------------------------------------------------------------------
+
+def test_max_sequence_length_band_alibi_sampled():
+    s = 1 << 20
+    w = W("BNSD", "bf16", (1, 1, s, 64), 1, 5000, pre_tokens=4096, next_tokens=0)
+    w.pse, w.pse_type = alibi_slopes(1), 2
+    res = run_gpu(w)
+    rows = sample_rows(w, 24, seed=1) + [(0, 0, s - 4097), (0, 0, 4095)]
+    compare_rows(w, res, rows)
+
+
+def test_max_tokens_varlen_causal_sampled():
+    lens = [262144, 131072, 393216, 262144]  # T = 1M
+    t = sum(lens)
+    w = W("TND", "bf16", (t, 1, 128), 1, 5100, actual_seq_q=cumulative(lens, False),
+          actual_seq_kv=cumulative(lens, False), next_tokens=0, sink=normal((1,), "f32", 5150))
+    res = run_gpu(w)
+    compare_rows(w, res, sample_rows(w, 12, seed=2))
+
+
+def test_max_sequences_varlen_sampled():
+    rng = np.random.default_rng(5200)
+    lens = [int(x) for x in rng.integers(0, 100, size=20000)]  # B = 20000, zero lengths included
+    t = sum(lens)
+    w = W("TND", "f16", (t, 2, 64), 2, 5210, actual_seq_q=cumulative(lens, False),
+          actual_seq_kv=cumulative(lens, False), next_tokens=0, sink=normal((2,), "f32", 5220))
+    assert "sm100_tcgen05" in plan_text(w)
+    res = run_gpu(w)
+    compare_rows(w, res, sample_rows(w, 48, seed=3))
+    # every row finite and written (zero-length sequences contribute no rows)
+    assert torch.isfinite(res[0].float()).all()
+
+
+def test_max_heads_gqa():
+    w = W("BNSD", "bf16", (1, 256, 200, 64), 256, 5300, kshape=(1, 8, 200, 64), next_tokens=0)
+    compare_full(w)
