@@ -17,7 +17,7 @@ scaleValue, preTockens/nextTockens, softmaxMax/softmaxSum):
     l_i     = sum_{keep} exp(s_ij - m_i) + [sink] exp(sink_n - m_i)
     o_i     = sum_{keep} exp(s_ij - m_i) v_j / l_i
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
   * pse is added after scaling, as the printed formula writes it;
   * the sink formula's S is this full transformed, masked score; the sink
     itself is neither scaled nor masked;
