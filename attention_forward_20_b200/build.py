@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfa_fwd.so")
-SOURCES = ["api.cpp", "fa_simt.cu", "fa_sm100.cu", "fa_static.cu", "fa_lse_merge.cu"]
+SOURCES = ["api.cpp", "fa_simt.cu", "fa_sm100.cu", "fa_static.cu", "fa_lse_merge.cu", "fa_upload.cu"]
 HEADERS = ["fa_params.h", "sm100_ptx.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

@@ -534,18 +534,17 @@ extern "C" fa_status fa_fwd(void* workspace, uint64_t workspaceSize, fa_executor
     char* ws = static_cast<char*>(workspace);
     fa::FaParams p = ex->p;
     if (!ex->cu.empty()) {
-        // Pageable source: the copy is staged before cudaMemcpyAsync returns,
-        // so the executor may be freed right after.
-        if (cudaMemcpyAsync(ws + ex->off_cu, ex->cu.data(), ex->cu.size() * sizeof(int64_t),
-                            cudaMemcpyHostToDevice, st) != cudaSuccess)
+        // Pageable source, staged before the call returns (or, under stream
+        // capture, carried by the graph), so the executor may be freed right after.
+        if (fa::upload_async(ws + ex->off_cu, ex->cu.data(), ex->cu.size() * sizeof(int64_t), st) != cudaSuccess)
             return done(FA_ERR_CUDA);
         p.cu_q = reinterpret_cast<const int64_t*>(ws + ex->off_cu);
         p.cu_kv = p.cu_q + (p.B + 1);
         if (p.pse_flat) p.pse_off = p.cu_q + 2 * (p.B + 1);
     }
     if (!ex->table.empty()) {
-        if (cudaMemcpyAsync(ws + ex->off_table, ex->table.data(), ex->table.size() * sizeof(int4),
-                            cudaMemcpyHostToDevice, st) != cudaSuccess)
+        if (fa::upload_async(ws + ex->off_table, ex->table.data(), ex->table.size() * sizeof(int4), st) !=
+            cudaSuccess)
             return done(FA_ERR_CUDA);
         p.table = reinterpret_cast<const int4*>(ws + ex->off_table);
     }

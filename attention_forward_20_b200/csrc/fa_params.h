@@ -156,5 +156,9 @@ uint64_t plan_sm100_schedule(FaParams& p, int num_sms, bool uniform, int item_kv
 // Encodes the Q/K/V (and rope) tensor maps for the tcgen05 kernel.
 cudaError_t make_sm100_tmaps(const FaParams& p, TmaSet* maps);
 uint64_t read_and_clear_device_error(cudaError_t* err);
+// Host-to-device copy of a small table: cudaMemcpyAsync, or, while `stream`
+// is being captured into a CUDA graph, copy kernels that carry the bytes in
+// their launch parameters (the graph keeps them; the host source may go).
+cudaError_t upload_async(void* dst, const void* src, size_t bytes, cudaStream_t stream);
 
 }  // namespace fa

@@ -225,10 +225,10 @@ extern "C" fa_status fa_fwd_varlen_static(
             p.n_items = p.table_len * p.Nq;
             bytes = kTableOffset + count * sizeof(int4);
         }
-        // Pageable source: staged before cudaMemcpyAsync returns, so the
-        // staging buffer may be reused once the lock is released.
-        if (cudaMemcpyAsync(dev, g_host_stage, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
-            return FA_ERR_CUDA;
+        // Pageable source: staged before the call returns (under stream
+        // capture the graph carries the bytes), so the staging buffer may be
+        // reused once the lock is released.
+        if (fa::upload_async(dev, g_host_stage, bytes, st) != cudaSuccess) return FA_ERR_CUDA;
     }
     p.cu_q = reinterpret_cast<const int64_t*>(dev + kCuOffset);
     p.cu_kv = p.cu_q + (nSeq + 1);

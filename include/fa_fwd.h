@@ -196,6 +196,11 @@ FA_API fa_status fa_fwd_get_workspace_size_v5(
  * returned (NULL allowed when that size is 0); it must stay untouched until
  * the stream work has finished.  The executor is consumed and freed on every
  * return path, success or error.
+ * The call may be captured into a CUDA graph (stream capture on `stream`):
+ * it then enqueues only capturable work, and the per-call tables (varlen
+ * offsets and work table) travel in the graph, so the graph replays
+ * correctly after the executor is gone; the workspace must stay allocated
+ * for as long as the graph is replayed.
  * Returns FA_SUCCESS, FA_ERR_PARAM_NULLPTR (executor NULL, or workspace NULL
  * with a nonzero size), FA_ERR_WORKSPACE or FA_ERR_CUDA. */
 FA_API fa_status fa_fwd(void* workspace, uint64_t workspaceSize, fa_executor* executor, void* stream);
