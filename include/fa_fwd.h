@@ -32,8 +32,10 @@
  * kernel merges.  Nothing in it has to be initialised by the caller.
  *
  * All floating-point accumulation is fp32.  Q·Kᵀ and P·V run on the tcgen05
- * tensor cores for fp16/bf16 inputs with head dim 64 or 128; fp32 inputs (and
- * any other head dim up to 256) run on an exact-FFMA CUDA-core kernel.
+ * tensor cores for fp16/bf16 inputs whose head dims (D, and Dv <= D) are
+ * multiples of 8 up to 256: zero-padded to 64 or 128 columns on a kernel that
+ * holds two 128-row query tiles, to 256 on a one-tile kernel.  fp32 inputs and
+ * other head dims up to 256 run on an exact-FFMA CUDA-core kernel.
  */
 #ifndef FA_FWD_H
 #define FA_FWD_H
@@ -161,8 +163,7 @@ FA_API fa_status fa_fwd_get_workspace_size(
  * the sizes and head counts of query / key and a head dim Dr of their own
  * (BSH/SBH: H = heads * Dr); D + Dr <= 256.  Not with realShift (the page:
  * incompatible), pseType 0 or 1.  A mismatch returns 561103.  Dr = 64 with
- * D = Dv in {64, 128} runs on the tensor cores; other sizes on the CUDA-core
- * kernel.
+ * D <= 128 runs on the tensor cores; other sizes on the CUDA-core kernel.
  *
  * qStartIdxOptional / kvStartIdxOptional: the start, in the whole sequence, of
  * the query and key/value chunk this call sees.  The band and an ALiBi bias
