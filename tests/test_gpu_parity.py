@@ -662,3 +662,54 @@ def test_max_sequences_varlen_sampled():
 def test_max_heads_gqa():
     w = W("BNSD", "bf16", (1, 256, 200, 64), 256, 5300, kshape=(1, 8, 200, 64), next_tokens=0)
     compare_full(w)
+
+
+# ---------------------------------------------------------------------------
+# Guard bands: outputs and statistics as views into larger buffers filled with
+# a sentinel (a guard zone before and after, padding columns in every row);
+# nothing outside the logical tensors may change.
+# ---------------------------------------------------------------------------
+
+def _guarded(shape, pad, dtype, sentinel=-7777.0, guard=4096):
+    padded = tuple(shape[:-1]) + (shape[-1] + pad,)
+    n = int(np.prod(padded))
+    base = torch.full((guard + n + guard,), sentinel, dtype=dtype, device="cuda")
+    view = base[guard:guard + n].view(padded)[..., :shape[-1]]
+    return base, view, (guard, n, padded)
+
+
+def _guards_intact(base, meta, width, sentinel=-7777.0):
+    guard, n, padded = meta
+    s = torch.tensor(sentinel, dtype=base.dtype, device="cuda")
+    assert torch.equal(base[:guard], s.expand(guard)), "write before the tensor"
+    assert torch.equal(base[guard + n:], s.expand(base.numel() - guard - n)), "write after the tensor"
+    pad_cols = base[guard:guard + n].view(padded)[..., width:]
+    assert torch.equal(pad_cols, s.expand_as(pad_cols)), "write into a row's padding"
+
+
+@pytest.mark.parametrize("case", ["dense_split_dv40", "varlen_ragged", "wide_dv136", "sbh_band"])
+def test_outputs_stay_inside_their_tensors(case):
+    dtype = torch.bfloat16
+    if case == "dense_split_dv40":
+        w = W("BNSD", "bf16", (1, 19, 2048, 48), 19, 5500, vshape=(1, 19, 2048, 40))
+        out_shape, st_shape = (1, 19, 2048, 40), (1, 19, 2048, 8)
+    elif case == "varlen_ragged":
+        lens = [129, 0, 300, 1, 255]
+        t = sum(lens)
+        w = W("TND", "bf16", (t, 3, 128), 3, 5510, actual_seq_q=cumulative(lens, False),
+              actual_seq_kv=cumulative(lens, False), next_tokens=0, sink=normal((3,), "f32", 5515))
+        out_shape, st_shape = (t, 3, 128), (3, t, 8)
+    elif case == "wide_dv136":
+        w = W("BNSD", "f16", (1, 2, 333, 256), 2, 5520, vshape=(1, 2, 333, 136), next_tokens=0)
+        out_shape, st_shape, dtype = (1, 2, 333, 136), (1, 2, 333, 8), torch.float16
+    else:
+        w = W("SBH", "bf16", (300, 2, 2 * 64), 2, 5530, pre_tokens=90, next_tokens=7)
+        out_shape, st_shape = (300, 2, 2 * 64), (2, 2, 300, 8)
+    ob, ov, om = _guarded(out_shape, 16, dtype)
+    mb, mv, mm = _guarded(st_shape, 8, torch.float32)
+    lb, lv, lm = _guarded(st_shape, 8, torch.float32)
+    res = run_gpu(w, out=ov, softmax_max=mv, softmax_sum=lv)
+    _guards_intact(ob, om, out_shape[-1])
+    _guards_intact(mb, mm, 8)
+    _guards_intact(lb, lm, 8)
+    compare_full(w, res=res)
