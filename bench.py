@@ -40,9 +40,11 @@ L2_FLUSH_BYTES = 256 << 20
 def workload_desc(w):
     lens = {"BNSD": (w.q.shape[0], w.q.shape[2]), "BSND": (w.q.shape[0], w.q.shape[1]),
             "BSH": (w.q.shape[0], w.q.shape[1]), "SBH": (w.q.shape[1], w.q.shape[0])}
-    d = w.q.shape[-1] if w.layout not in ("BSH", "SBH") else w.q.shape[-1] // w.head_num
+    d, dv = head_dims(w)
     cfg = {"workload": f"{w.name} {w.layout} {w.dtype}", "layout": w.layout, "dtype": w.dtype,
            "heads": w.head_num, "head_dim": d}
+    if dv != d:
+        cfg["value_head_dim"] = dv
     if w.layout == "TND":
         cfg.update(tokens=w.q.shape[0], lengths=w.extra.get("lengths"))
     else:
@@ -57,11 +59,19 @@ def workload_desc(w):
     return cfg
 
 
+def head_dims(w):
+    """(query/key head dim, value head dim) of workload w."""
+    if w.layout in ("BSH", "SBH"):
+        d = w.q.shape[-1] // w.head_num
+        return d, w.v.shape[-1] // (w.k.shape[-1] // d)
+    return w.q.shape[-1], w.v.shape[-1]
+
+
 def tile_flops(w):
-    """4 * D * (query-row x key pairs), counted over every 128x128 tile that
-    holds at least one kept pair (the headline rule), and the exact kept-pair
-    FLOPs beside it."""
-    d = w.q.shape[-1] if w.layout not in ("BSH", "SBH") else w.q.shape[-1] // w.head_num
+    """(2*D + 2*Dv) * (query-row x key pairs), counted over every 128x128 tile
+    that holds at least one kept pair (the headline rule), and the exact
+    kept-pair FLOPs beside it (4*D per pair when Dv = D)."""
+    d, dv = head_dims(w)
     if w.layout == "TND":
         lens_q = np.diff([0] + list(w.actual_seq_q))
         lens_k = np.diff([0] + list(w.actual_seq_kv))
@@ -87,7 +97,8 @@ def tile_flops(w):
                     tiles += 128 * 128
                     exact += int(kept)
     heads = w.head_num
-    return 4.0 * d * tiles * heads, 4.0 * d * exact * heads
+    per_pair = 2.0 * d + 2.0 * dv
+    return per_pair * tiles * heads, per_pair * exact * heads
 
 
 def sources_sha():
@@ -199,6 +210,24 @@ def alibi_bias_on_device(slopes, seq, first_row, dtype, dev):
     return bias
 
 
+def with_head_dims(w, d, dv):
+    """Workload w with query/key head dim d and value head dim dv: same layout,
+    sizes, masks and seeds, inputs redrawn N(0,1), scale d^-0.5."""
+    def shaped(t, heads, hd):
+        if w.layout in ("BSH", "SBH"):
+            return tuple(t.shape[:2]) + (heads * hd,)
+        return tuple(t.shape[:-1]) + (hd,)
+    d0 = w.q.shape[-1] // w.head_num if w.layout in ("BSH", "SBH") else w.q.shape[-1]
+    n_kv = w.k.shape[-1] // d0 if w.layout in ("BSH", "SBH") else None
+    seed = 7000 + 17 * w.number
+    w.q = normal(shaped(w.q, w.head_num, d), w.dtype, seed)
+    w.k = normal(shaped(w.k, n_kv, d), w.dtype, seed + 1)
+    w.v = normal(shaped(w.v, n_kv, dv), w.dtype, seed + 2)
+    w.scale = d ** -0.5
+    w.name = f"{w.name}_d{d}" + (f"_dv{dv}" if dv != d else "")
+    return w
+
+
 def rope_tensors(w, dr, seed):
     """queryRope / keyRope for workload w: the query's / key's layout and sizes, head dim dr."""
     def shaped(t, heads):
@@ -224,7 +253,7 @@ def time_oracle(w, budget_s, max_heads=None, rope=None):
     `budget_s` seconds have passed; returns (flops done, seconds, heads done).
     rope: (queryRope, keyRope) host tensors or None."""
     from oracle import ref
-    d = w.q.shape[-1] if w.layout not in ("BSH", "SBH") else w.q.shape[-1] // w.head_num
+    d, dv = head_dims(w)
     dr = 0
     if rope is not None:
         dr = rope[0].shape[-1] if w.layout not in ("BSH", "SBH") else rope[0].shape[-1] // w.head_num
@@ -232,7 +261,7 @@ def time_oracle(w, budget_s, max_heads=None, rope=None):
         krh = ref.heads_view(rope[1].double().numpy(), w.layout, dr)
     qh = ref.heads_view(w.q.double().numpy(), w.layout, d)
     kh = ref.heads_view(w.k.double().numpy(), w.layout, d)
-    vh = ref.heads_view(w.v.double().numpy(), w.layout, d)
+    vh = ref.heads_view(w.v.double().numpy(), w.layout, dv)
     n_kv = kh.shape[1]
     group = w.head_num // n_kv
     sink = None if w.sink is None else w.sink.double().numpy()
@@ -262,7 +291,7 @@ def time_oracle(w, budget_s, max_heads=None, rope=None):
                          pre_tokens=w.pre_tokens, next_tokens=w.next_tokens,
                          sink=None if sink is None else sink[n], q_rope=qr, k_rope=kr)
         secs += time.perf_counter() - t0
-        flops += (4.0 * d + 2.0 * dr) * q.shape[0] * k.shape[0]
+        flops += (2.0 * d + 2.0 * dv + 2.0 * dr) * q.shape[0] * k.shape[0]
         heads += 1
         if secs >= budget_s:
             break
@@ -355,6 +384,9 @@ def main():
                          "then fa_lse_merge (dense layouts)")
     ap.add_argument("--pse", default="slopes", choices=["slopes", "dense", "compressed"],
                     help="ALiBi workloads: slopes in-kernel, a materialised [1,N,S,S] bias, or its last 1024 rows")
+    ap.add_argument("--head-dim", type=int, default=0,
+                    help="the workload with this query/key head dim (fresh N(0,1) inputs, scale D^-0.5)")
+    ap.add_argument("--value-head-dim", type=int, default=0, help="with --head-dim: the value head dim (default D)")
     ap.add_argument("--rope", type=int, default=0,
                     help="bf16 workloads: add queryRope/keyRope of this head dim (N(0,1), seeded)")
     args = ap.parse_args()
@@ -377,7 +409,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     # each rank: its own shard (seed offset by rank) of the workload's batch
-    w = shard_workload(build(args.workload), rank)
+    w = build(args.workload)
+    if args.head_dim:
+        w = with_head_dims(w, args.head_dim, args.value_head_dim or args.head_dim)
+    w = shard_workload(w, rank)
     flops_tiles, flops_exact = tile_flops(w)
     q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
     kw = fa_kwargs(w, dev)
@@ -387,10 +422,10 @@ def main():
             raise SystemExit("--rope needs a bf16 workload (queryRope/keyRope are BFLOAT16 only)")
         rope = rope_tensors(w, args.rope, seed=9100 + rank)
         kw["query_rope"], kw["key_rope"] = rope[0].to(dev), rope[1].to(dev)
-        # S = Q K^T + Qr Kr^T: 2*(D + Dr) + 2*Dv FLOPs per kept pair instead of 4*D
-        d = w.q.shape[-1] // w.head_num if w.layout in ("BSH", "SBH") else w.q.shape[-1]
-        flops_tiles *= (4.0 * d + 2.0 * args.rope) / (4.0 * d)
-        flops_exact *= (4.0 * d + 2.0 * args.rope) / (4.0 * d)
+        # S = Q K^T + Qr Kr^T: 2*(D + Dr) + 2*Dv FLOPs per kept pair
+        d, dv = head_dims(w)
+        flops_tiles *= (2.0 * d + 2.0 * dv + 2.0 * args.rope) / (2.0 * d + 2.0 * dv)
+        flops_exact *= (2.0 * d + 2.0 * dv + 2.0 * args.rope) / (2.0 * d + 2.0 * dv)
     bias_bytes = 0
     if args.pse != "slopes" and w.pse_type == 2:
         # the same ALiBi bias, materialised in the query dtype and resident in HBM
@@ -400,8 +435,8 @@ def main():
         kw["real_shift"] = alibi_bias_on_device(w.pse.double().numpy(), seq, first, q.dtype, dev)
         kw["pse_type"] = 1
         # bias bytes the kernel reads: one 128x128 block per counted tile-block
-        d = w.q.shape[-1] // w.head_num if w.layout in ("BSH", "SBH") else w.q.shape[-1]
-        bias_bytes = flops_tiles / (4.0 * d) * q.element_size()
+        d, dv = head_dims(w)
+        bias_bytes = flops_tiles / (2.0 * d + 2.0 * dv) * q.element_size()
     out, smax, ssum = fa.fa_fwd(q, k, v, **kw)
     launches_per_step = kernels_per_call(fa, q, k, v, kw)
     if args.kv_chunks > 1:
