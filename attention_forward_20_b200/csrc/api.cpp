@@ -459,6 +459,9 @@ extern "C" fa_status fa_fwd_get_workspace_size_v5(
         } else {
             p.n_qb = (int32_t)((max_q + kQBlock - 1) / kQBlock);
             p.items_per_n_block = (int32_t)(B * qv.N);
+            // 16 heads of K/V at D <= 128 (2 MB each at 4096 keys) stay in L2;
+            // the one-tile kernel for larger D streams them twice per item, 4 heads
+            p.head_group = qv.D > 128 ? 4 : 16;
             p.n_items = p.n_qb * p.items_per_n_block;
         }
         // Equal-cost items (every query block touches the same number of key

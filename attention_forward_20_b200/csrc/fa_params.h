@@ -53,6 +53,7 @@ struct FaParams {
     int32_t n_items;            // work items of (b, n, 256-row query block)
     int32_t n_qb;               // query blocks per (b, n) for the dense layouts
     int32_t items_per_n_block;  // dense: B * Nq
+    int32_t head_group;         // dense: heads whose items run together, so that their K/V stay in L2
     const int4* table;          // TND: {b, qb, q_len, kv_len} per (sequence, block), heads implied
     int32_t table_len;
     int32_t neg_scale;          // scaleValue < 0: the kernel negates K inside the MMA

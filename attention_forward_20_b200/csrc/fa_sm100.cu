@@ -58,7 +58,6 @@ constexpr uint32_t kSoftmaxRegs = 216;  // per thread, softmax warpgroups (setma
 constexpr uint32_t kOtherRegs = 72;     // per thread, producer/MMA warpgroup
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kHeadGroup = 16;  // heads whose items run together, so their K/V stay in L2
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kRescaleThreshold = 8.0f;
@@ -115,7 +114,7 @@ struct TicketSlots {
 };
 
 // Work item -> (batch, head, query block).  Dense layouts: groups of
-// kHeadGroup heads; inside a group the query blocks go from the last (the
+// p.head_group heads; inside a group the query blocks go from the last (the
 // most keys under a causal band) to the first, heads fastest.  TND: the host
 // table lists (sequence, block) longest first; heads fastest.
 __device__ __forceinline__ Item decode_item(const FaParams& p, int item) {
@@ -132,12 +131,13 @@ __device__ __forceinline__ Item decode_item(const FaParams& p, int item) {
         it.kv_off = p.cu_kv[it.b];
     } else {
         const int bn_total = p.B * p.Nq;
-        const int per_group = kHeadGroup * p.n_qb;
+        const int hg = p.head_group;
+        const int per_group = hg * p.n_qb;
         const int g = item / per_group;
         const int within = item - g * per_group;
-        const int g_heads = min(kHeadGroup, bn_total - g * kHeadGroup);
+        const int g_heads = min(hg, bn_total - g * hg);
         const int level = within / g_heads;
-        const int bn = g * kHeadGroup + (within - level * g_heads);
+        const int bn = g * hg + (within - level * g_heads);
         it.qb = p.n_qb - 1 - level;
         it.b = bn / p.Nq;
         it.n = bn - it.b * p.Nq;
