@@ -360,11 +360,11 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
     for (int s = 0; s < C::kStages; ++s) {
         if ((uint32_t)s < kv_fill) {
             const uint32_t last = kv_fill - 1 - ((kv_fill - 1 - s) % C::kStages);
-            mbar_wait(&bars.kv_full[s], (last / C::kStages) & 1, abort, kSiteDrain);
+            mbar_wait_drain(&bars.kv_full[s], (last / C::kStages) & 1, abort, kSiteDrain);
         }
     }
     for (int t = 0; t < 2; ++t)
-        if (q_fill[t]) mbar_wait(&bars.q_full[t], (q_fill[t] - 1) & 1, abort, kSiteDrain);
+        if (q_fill[t]) mbar_wait_drain(&bars.q_full[t], (q_fill[t] - 1) & 1, abort, kSiteDrain);
 }
 
 // ---------------------------------------------------------------------------
@@ -480,7 +480,7 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* s
     }
     // Drain: every MMA this warp issued completes before TMEM is freed.
     commit(&bars.drain);
-    warp_wait(&bars.drain, 0, abort, kSiteDrain);
+    __all_sync(0xffffffffu, mbar_wait_drain(&bars.drain, 0, abort, kSiteDrain));
 }
 
 // ---------------------------------------------------------------------------
@@ -567,10 +567,10 @@ __device__ void run_producer_wide(const FaParams& p, const CUtensorMap* tq, cons
     for (int sl = 0; sl < kWideSlots; ++sl) {
         if ((uint32_t)sl < fill) {
             const uint32_t last = fill - 1 - ((fill - 1 - sl) % kWideSlots);
-            mbar_wait(&bars.kv_full[sl], (last / kWideSlots) & 1, abort, kSiteDrain);
+            mbar_wait_drain(&bars.kv_full[sl], (last / kWideSlots) & 1, abort, kSiteDrain);
         }
     }
-    if (q_fill) mbar_wait(&bars.q_full[0], (q_fill - 1) & 1, abort, kSiteDrain);
+    if (q_fill) mbar_wait_drain(&bars.q_full[0], (q_fill - 1) & 1, abort, kSiteDrain);
 }
 
 template <typename T>
@@ -663,7 +663,7 @@ __device__ void run_mma_wide(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barri
         }
     }
     commit(&bars.drain);
-    warp_wait(&bars.drain, 0, abort, kSiteDrain);
+    __all_sync(0xffffffffu, mbar_wait_drain(&bars.drain, 0, abort, kSiteDrain));
 }
 
 // ---------------------------------------------------------------------------

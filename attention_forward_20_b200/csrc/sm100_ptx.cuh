@@ -81,6 +81,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// Drain waits: copies and MMAs that the CTA has already issued must complete
+// before it frees TMEM or exits, after an abort as well, so these ignore
+// *abort; they are bounded by kDrainLimitNs (work in flight lands within
+// microseconds) and record `site` if that runs out.
+constexpr uint64_t kDrainLimitNs = 200000000ull;  // 200 ms
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, volatile int* abort, int site) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 31u) == 0 && (it >= kWaitLimitIters || globaltimer_ns() - t0 > kDrainLimitNs)) {
+            atomicCAS(const_cast<int*>(abort), 0, site);
+            return false;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast.  `tmap` is the generic address of
 // a __grid_constant__ CUtensorMap kernel parameter.
