@@ -273,7 +273,12 @@ FA_API fa_status fa_device_error(uint64_t* detail);
  * device, with that device current); make that first call before any stream
  * capture.  Every call overwrites the part of the array it reads, so nothing
  * needs clearing, but calls whose work overlaps on the GPU (other streams,
- * other host threads) race on the shared array.
+ * other host threads) race on the shared array.  Under stream capture the
+ * offsets and table travel in the graph (copy kernels that carry the bytes in
+ * their launch parameters), so each replay writes its own table back into the
+ * array first; replays, like calls, must not overlap on the GPU.
+ * fp16/bf16 with head dims up to 128 run on the tensor cores, the rest on the
+ * CUDA-core kernel.
  *
  * Returns FA_SUCCESS, FA_ERR_PARAM_NULLPTR, FA_ERR_PARAM_INVALID,
  * FA_ERR_INNER_NULLPTR or FA_ERR_CUDA. */
