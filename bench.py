@@ -27,7 +27,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from workloads import build, normal  # noqa: E402
+from workloads import build, normal, cumulative  # noqa: E402
 
 METRIC = "FA forward TFLOP/s and % of B200 dense BF16/FP16 peak (1 GPU)"
 UNIT = "TFLOP/s"
@@ -339,6 +339,40 @@ def whole_job_tflops(flops_per_rank, world, ms_per_step):
     return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
 
 
+def step_stats(times_ms):
+    """Median, min, p90 and mean of per-step times (ms)."""
+    t = np.asarray(times_ms, dtype=np.float64)
+    return {"median": float(np.median(t)), "min": float(t.min()), "p90": float(np.percentile(t, 90)),
+            "mean": float(t.mean())}
+
+
+def time_oracle_single_thread(w, rope=None):
+    """The oracle on one whole (batch, head) of w with one BLAS thread: (TFLOP/s, seconds)."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        fl, secs, _ = time_oracle(w, 0.0, max_heads=1, rope=rope)
+    return fl / secs / 1e12, secs
+
+
+def with_lengths(w, lengths):
+    """Varlen (TND) workload w with other sequence lengths: inputs redrawn with
+    the same seeds at T = sum(lengths), q and kv lengths equal."""
+    if w.layout != "TND":
+        raise SystemExit("--lengths applies to the TND workload")
+    lens = [int(x) for x in lengths]
+    t = sum(lens)
+    seed = 1000 * w.number
+    w.q = normal((t,) + tuple(w.q.shape[1:]), w.dtype, seed + 1)
+    w.k = normal((t,) + tuple(w.k.shape[1:]), w.dtype, seed + 2)
+    w.v = normal((t,) + tuple(w.v.shape[1:]), w.dtype, seed + 3)
+    w.actual_seq_q = cumulative(lens, False)
+    w.actual_seq_kv = cumulative(lens, False)
+    w.extra["lengths"] = lens
+    w.extra["cu_seqlens"] = cumulative(lens, True)
+    w.name = w.name + "_" + "_".join(str(x) for x in lens)
+    return w
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -387,6 +421,8 @@ def main():
     ap.add_argument("--head-dim", type=int, default=0,
                     help="the workload with this query/key head dim (fresh N(0,1) inputs, scale D^-0.5)")
     ap.add_argument("--value-head-dim", type=int, default=0, help="with --head-dim: the value head dim (default D)")
+    ap.add_argument("--lengths", default="",
+                    help="TND workload: comma-separated sequence lengths instead of the seeded ones")
     ap.add_argument("--rope", type=int, default=0,
                     help="bf16 workloads: add queryRope/keyRope of this head dim (N(0,1), seeded)")
     args = ap.parse_args()
@@ -410,6 +446,8 @@ def main():
 
     # each rank: its own shard (seed offset by rank) of the workload's batch
     w = build(args.workload)
+    if args.lengths:
+        w = with_lengths(w, args.lengths.split(","))
     if args.head_dim:
         w = with_head_dims(w, args.head_dim, args.value_head_dim or args.head_dim)
     w = shard_workload(w, rank)
@@ -438,6 +476,8 @@ def main():
         d, dv = head_dims(w)
         bias_bytes = flops_tiles / (2.0 * d + 2.0 * dv) * q.element_size()
     out, smax, ssum = fa.fa_fwd(q, k, v, **kw)
+    if not (bool(torch.isfinite(out).all()) and not bool(torch.isnan(smax).any())):
+        raise SystemExit("first forward gave non-finite outputs")
     launches_per_step = kernels_per_call(fa, q, k, v, kw)
     if args.kv_chunks > 1:
         launches_per_step = args.kv_chunks * launches_per_step + 1  # chunk forwards + the merge (upper bound)
@@ -502,7 +542,8 @@ def main():
         torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
-    kernel_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    step_times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kernel_ms = sum(step_times)
     status, word = fa.device_error()
     if status != 0:
         raise SystemExit(f"kernel error word {word:#x}")
@@ -578,6 +619,7 @@ def main():
     peak, peak_src = load_peak()
     traffic = load_traffic(w.name) if args.pse == "slopes" and not args.rope else None
     fl, secs, heads = time_oracle(w, args.cpu_budget, rope=rope)
+    st_value, st_secs = time_oracle_single_thread(w, rope=rope)
     cpu_value = fl / secs / 1e12
     desc = workload_desc(w)
     merge_line = None
@@ -608,10 +650,13 @@ def main():
         "cpu_baseline": {"value": cpu_value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                          "sample": f"{heads} whole (batch, head) pairs of the workload, float64 NumPy, "
                                    f"{secs:.1f} s" + ("" if args.pse == "slopes" else
-                                                      " (bias from the slopes, the same values in float64)")},
+                                                      " (bias from the slopes, the same values in float64)"),
+                         "single_thread": {"value": st_value, "unit": UNIT,
+                                           "sample": f"one whole (batch, head), one BLAS thread, {st_secs:.1f} s"}},
         "e2e": {"value": whole_job_tflops(flops_tiles, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "pipeline": "copy in / compute / copy out on three streams, two buffer sets"},
+        "step_ms": step_stats(step_times),
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clocks.summary(),
     }

@@ -105,3 +105,24 @@ def test_varlen_flops_sum_over_sequences():
     want_tiles = sum(_brute_tiles(n, n, 10**6, 0)[0] for n in lens if n)
     assert tiles == 4.0 * 64 * want_tiles * 128 * 128 * 2
     assert np.isfinite(tiles)
+
+
+def test_step_stats():
+    st = bench.step_stats([1.0, 2.0, 3.0, 4.0, 10.0])
+    assert st["median"] == 3.0 and st["min"] == 1.0 and st["mean"] == 4.0
+    assert 4.0 <= st["p90"] <= 10.0
+
+
+def test_with_lengths_rebuilds_the_varlen_workload():
+    w = bench.with_lengths(build(4), ["2048", "2048", "2048", "2048"])
+    assert w.q.shape == (8192, 24, 128) and w.actual_seq_q == [2048, 4096, 6144, 8192]
+    assert w.extra["cu_seqlens"] == [0, 2048, 4096, 6144, 8192] and w.name.endswith("_2048_2048_2048_2048")
+    assert w.actual_seq_kv == w.actual_seq_q
+    # the default lengths' inputs come from the same seeds
+    w0 = build(4)
+    assert bench.with_lengths(build(4), w0.extra["lengths"]).q.float().sum() == w0.q.float().sum()
+
+
+def test_single_thread_oracle_time():
+    value, secs = bench.time_oracle_single_thread(build(1))
+    assert value > 0 and secs > 0
