@@ -504,3 +504,55 @@ def test_limits_rejected_one_past():
     t = torch.zeros(20000, 1, 8, dtype=torch.float16)
     cum = list(range(1, 20001))
     assert plan(t, t, t, input_layout="TND", head_num=1, actual_seq_qlen=cum, actual_seq_kvlen=cum)[0] == 0
+
+
+def test_header_is_plain_c_and_stage_one_runs_from_c(built, tmp_path):
+    """A C99 program compiles against include/fa_fwd.h (no C++ or torch types
+    in the interface), links libfa_fwd.so, plans a dense BNSD call and a bad
+    layout, and frees the plan; stage 1 touches no device memory."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "stage1.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "fa_fwd.h"
+
+static fa_tensor bnsd(int32_t dtype, int64_t b, int64_t n, int64_t s, int64_t d, void* data) {
+    fa_tensor t;
+    memset(&t, 0, sizeof t);
+    t.data = data; t.dtype = dtype; t.ndim = 4;
+    t.shape[0] = b; t.shape[1] = n; t.shape[2] = s; t.shape[3] = d;
+    t.strides[3] = 1; t.strides[2] = d; t.strides[1] = s * d; t.strides[0] = n * s * d;
+    return t;
+}
+
+int main(void) {
+    void* fake = (void*)(uintptr_t)0x100000; /* never dereferenced by stage 1 */
+    fa_tensor q = bnsd(FA_F16, 2, 4, 1000, 128, fake), o = q;
+    fa_tensor st = bnsd(FA_F32, 2, 4, 1000, 8, fake);
+    uint64_t ws = 0;
+    fa_executor* ex = NULL;
+    fa_status s = fa_fwd_get_workspace_size(&q, &q, &q, NULL, NULL, NULL, NULL, 0, NULL, 0, 0.088, 1.0,
+                                            INT64_MAX, 0, 4, "BNSD", 0, 0, 0, "", &st, &st, &o, &ws, &ex);
+    if (s != FA_SUCCESS || ex == NULL) return 1;
+    printf("%s\n", fa_executor_describe(ex));
+    fa_executor_destroy(ex);
+    s = fa_fwd_get_workspace_size(&q, &q, &q, NULL, NULL, NULL, NULL, 0, NULL, 0, 0.088, 1.0,
+                                  INT64_MAX, 0, 4, "XYZ", 0, 0, 0, "", &st, &st, &o, &ws, &ex);
+    if (s != FA_ERR_PARAM_INVALID || ex != NULL) return 2;
+    printf("%s\n", fa_status_string(s));
+    return 0;
+}
+''')
+    lib = os.path.join(ROOT, "attention_forward_20_b200", "libfa_fwd.so")
+    exe = tmp_path / "stage1"
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                         str(src), lib, "-o", str(exe), f"-Wl,-rpath,{os.path.dirname(lib)}"],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
+    assert "kernel=sm100_tcgen05" in run.stdout and "FA_ERR_PARAM_INVALID" in run.stdout
