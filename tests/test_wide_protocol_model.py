@@ -117,6 +117,8 @@ def run(tiles, v_halves, seed):
                     vs.append((yield from take(("V", j, h))))
                 yield ("wait", f"p_full{buf}", p_cnt[buf] & 1, p_cnt[buf])
                 p_cnt[buf] += 1
+                for h, s in enumerate(vs):
+                    assert ring.get(s) == ("V", j, h), ("P·V reads a slot that no longer holds V", j, h)
                 log.append(("PV", j, buf))
                 b("pv_done").arrive()
                 for s in vs:
