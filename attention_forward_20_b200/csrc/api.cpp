@@ -122,6 +122,42 @@ int64_t kv_blocks_for_tile(int64_t r0, int64_t q_len, int64_t kv_len, int64_t pr
 
 }  // namespace
 
+namespace fa {
+
+int64_t varlen_table_len(const int64_t* cu_q, int64_t B) {
+    int64_t n = 0;
+    for (int64_t b = 0; b < B; ++b) n += (cu_q[b + 1] - cu_q[b] + kQBlock - 1) / kQBlock;
+    return n;
+}
+
+void build_varlen_table(const int64_t* cu_q, const int64_t* cu_kv, int64_t B, int64_t pre, int64_t next,
+                        VarlenEntry* scratch, int4* out) {
+    int64_t count = 0;
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t ql = cu_q[b + 1] - cu_q[b];
+        const int64_t kl = cu_kv[b + 1] - cu_kv[b];
+        for (int64_t qb = 0; qb * kQBlock < ql; ++qb) {
+            const int64_t cost = kv_blocks_for_tile(qb * kQBlock, ql, kl, pre, next) +
+                                 kv_blocks_for_tile(qb * kQBlock + 128, ql, kl, pre, next);
+            scratch[count] = {cost, count, make_int4((int)b, (int)qb, (int)ql, (int)kl)};
+            ++count;
+        }
+    }
+    // a total order (cost, then position), so an in-place sort gives one result
+    std::sort(scratch, scratch + count, [](const VarlenEntry& a, const VarlenEntry& c) {
+        return a.cost != c.cost ? a.cost > c.cost : a.order < c.order;
+    });
+    for (int64_t e = 0; e < count; ++e) out[e] = scratch[e].e;
+}
+
+bool tma_dim_ok(int64_t stride, int64_t size) {
+    if (size == 1) return true;
+    const int64_t bytes = stride * 2;
+    return stride > 0 && bytes % 16 == 0 && bytes < (int64_t(1) << 40);
+}
+
+}  // namespace fa
+
 extern "C" fa_status fa_fwd_get_workspace_size_v5(
     const fa_tensor* query, const fa_tensor* queryRope, const fa_tensor* key, const fa_tensor* keyRope,
     const fa_tensor* value,
@@ -406,11 +442,7 @@ extern "C" fa_status fa_fwd_get_workspace_size_v5(
     // tcgen05 needs fp16/bf16, D <= 256, and TMA-legal operands:
     // 16-byte aligned bases and, for every dimension longer than 1, a positive
     // byte stride that is a multiple of 16 and below 2^40.
-    auto tma_dim_ok = [](int64_t stride, int64_t size) {
-        if (size == 1) return true;
-        const int64_t bytes = stride * 2;
-        return stride > 0 && bytes % 16 == 0 && bytes < (int64_t(1) << 40);
-    };
+    using fa::tma_dim_ok;
     bool tma_ok = aligned16(p.q) && aligned16(p.k) && aligned16(p.v);
     const int64_t qB = L == L_TND ? 1 : B;
     tma_ok = tma_ok && tma_dim_ok(p.q_s, qv.S) && tma_dim_ok(p.q_n, qv.N) && tma_dim_ok(p.q_b, qB);
@@ -438,20 +470,11 @@ extern "C" fa_status fa_fwd_get_workspace_size_v5(
     }
     if (sm100) {
         if (L == L_TND) {
-            struct Entry { int64_t cost; int4 e; };
-            std::vector<Entry> entries;
-            for (int64_t b = 0; b < B; ++b) {
-                const int64_t ql = ex->cu[b + 1] - ex->cu[b];
-                const int64_t kl = ex->cu[B + 2 + b] - ex->cu[B + 1 + b];
-                for (int64_t qb = 0; qb * kQBlock < ql; ++qb) {
-                    const int64_t cost = kv_blocks_for_tile(qb * kQBlock, ql, kl, pre_c, next_c) +
-                                         kv_blocks_for_tile(qb * kQBlock + 128, ql, kl, pre_c, next_c);
-                    entries.push_back({cost, make_int4((int)b, (int)qb, (int)ql, (int)kl)});
-                }
-            }
-            std::stable_sort(entries.begin(), entries.end(),
-                             [](const Entry& a, const Entry& c) { return a.cost > c.cost; });
-            for (const auto& e : entries) ex->table.push_back(e.e);
+            const int64_t len = fa::varlen_table_len(ex->cu.data(), B);
+            std::vector<fa::VarlenEntry> scratch(len);
+            ex->table.resize(len);
+            fa::build_varlen_table(ex->cu.data(), ex->cu.data() + B + 1, B, pre_c, next_c, scratch.data(),
+                                   ex->table.data());
             ex->off_table = off;
             off += ex->table.size() * sizeof(int4);
             p.table_len = (int32_t)ex->table.size();

@@ -146,6 +146,26 @@ struct TmaSet {
     TmaDesc q, k, v, qr, kr;
 };
 
+// Varlen work table of the tcgen05 kernels: one entry {b, qb, q_len, kv_len}
+// per (sequence b, 256-row query block qb), longest first -- by the number of
+// 128-key blocks the block's two query tiles touch under the band
+// -pre <= j - i <= next -- with ties in (sequence, block) order.  cu_q and
+// cu_kv are cumulative lengths with a leading 0 (B + 1 entries each).
+struct VarlenEntry {
+    int64_t cost;
+    int64_t order;
+    int4 e;
+};
+int64_t varlen_table_len(const int64_t* cu_q, int64_t B);
+// Writes varlen_table_len() entries to `out`, using `scratch` (as many
+// VarlenEntry) for the sort; allocates nothing.
+void build_varlen_table(const int64_t* cu_q, const int64_t* cu_kv, int64_t B, int64_t pre, int64_t next,
+                        VarlenEntry* scratch, int4* out);
+// A tensor-map dimension of `size` elements with an element stride of
+// `stride` (16-bit elements): legal for TMA when the size is 1, or the byte
+// stride is positive, a multiple of 16 and below 2^40.
+bool tma_dim_ok(int64_t stride, int64_t size);
+
 cudaError_t launch_simt(const FaParams& p, cudaStream_t stream);
 cudaError_t launch_sm100(const FaParams& p, const TmaSet& maps, int num_sms, cudaStream_t stream);
 // Schedule of the tcgen05 kernel (fills grid, n_whole, n_pieces, n_tickets

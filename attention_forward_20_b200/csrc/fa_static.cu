@@ -35,10 +35,15 @@ namespace {
 constexpr int64_t kStaticMaxSeqs = 2048;
 constexpr int64_t kStaticMaxBlocks = (int64_t(1) << 20) / 256 + kStaticMaxSeqs;
 constexpr size_t kCuOffset = 256;  // [0, 256): the tcgen05 kernel's ticket counter
-constexpr size_t kCuBytes = 2 * (kStaticMaxSeqs + 1) * sizeof(int64_t);
-constexpr size_t kTableOffset = (kCuOffset + kCuBytes + 255) & ~size_t(255);
-constexpr size_t kScratchBytes = kTableOffset + kStaticMaxBlocks * sizeof(int4);
+constexpr size_t kMaxCuBytes = 2 * (kStaticMaxSeqs + 1) * sizeof(int64_t);
+constexpr size_t kScratchBytes = ((kCuOffset + kMaxCuBytes + 255) & ~size_t(255)) + kStaticMaxBlocks * sizeof(int4);
 constexpr int kMaxDevices = 64;
+
+// Offset of the work table for a call with nSeq sequences: right after that
+// call's offsets, 256-byte aligned (at most kScratchBytes - the table).
+size_t table_offset(int64_t nSeq) {
+    return (kCuOffset + 2 * (nSeq + 1) * sizeof(int64_t) + 255) & ~size_t(255);
+}
 
 // The scratch.  In host code this name is only a stand-in for the symbol, not
 // a device address; host code must use the address from cudaGetSymbolAddress.
@@ -46,26 +51,29 @@ static __device__ __align__(256) unsigned char g_static_scratch[kScratchBytes];
 
 // Host staging for the offsets and table (static storage, one caller at a time).
 static unsigned char g_host_stage[kScratchBytes];
+static fa::VarlenEntry g_sort_stage[kStaticMaxBlocks];
 static std::mutex g_stage_mutex;
 
 static void* g_scratch_ptr[kMaxDevices];
-static cudaError_t g_scratch_err[kMaxDevices];
-static std::once_flag g_scratch_once[kMaxDevices];
+static std::mutex g_scratch_mutex[kMaxDevices];
 
-// Device address of the scratch on the current device, looked up once per
-// device (the first call on a device does the lookup).
+// Device address of the scratch on the current device.  A successful lookup
+// is kept for the device; a failed one (a transient error, or a first call
+// made while a stream is being captured) is not, so the next call tries again.
 cudaError_t scratch_address(void** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::call_once(g_scratch_once[dev], [dev] {
+    std::lock_guard<std::mutex> lock(g_scratch_mutex[dev]);
+    if (g_scratch_ptr[dev] == nullptr) {
         void* ptr = nullptr;
-        g_scratch_err[dev] = cudaGetSymbolAddress(&ptr, g_static_scratch);
+        e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+        if (e != cudaSuccess) return e;
         g_scratch_ptr[dev] = ptr;
-    });
+    }
     *out = g_scratch_ptr[dev];
-    return g_scratch_err[dev];
+    return cudaSuccess;
 }
 
 bool tnd_view(const fa_tensor* t, int64_t* T, int64_t* N, int64_t* D, int64_t* st, int64_t* sn) {
@@ -79,20 +87,6 @@ bool tnd_view(const fa_tensor* t, int64_t* T, int64_t* N, int64_t* D, int64_t* s
     *sn = t->strides[1];
     return true;
 }
-
-int64_t blocks_for_tile(int64_t r0, int64_t q_len, int64_t kv_len, int64_t pre, int64_t next) {
-    const int64_t r1 = std::min(q_len, r0 + 128) - 1;
-    if (r1 < r0 || kv_len <= 0) return 0;
-    const int64_t lo = std::max<int64_t>(0, r0 - pre);
-    const int64_t hi = std::min<int64_t>(kv_len - 1, r1 + next);
-    return hi < lo ? 0 : hi / 128 - lo / 128 + 1;
-}
-
-struct CostEntry {
-    int64_t cost;
-    int4 e;
-};
-static CostEntry g_cost_stage[kStaticMaxBlocks];
 
 }  // namespace
 
@@ -175,10 +169,10 @@ extern "C" fa_status fa_fwd_varlen_static(
     auto aligned32 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 31u) == 0; };
     p.o_vec32 = aligned32(p.o) && p.o_n % 16 == 0 && p.o_s % 16 == 0;
     p.st_vec32 = aligned32(p.smax) && aligned32(p.ssum) && p.st_n % 8 == 0 && p.st_s % 8 == 0;
-    auto tma_dim_ok = [](int64_t stride, int64_t size) {
-        return size == 1 || (stride > 0 && (stride * 2) % 16 == 0 && stride * 2 < (int64_t(1) << 40));
-    };
-    const bool sm100 = (dt == FA_F16 || dt == FA_BF16) && D <= 128 && D % 8 == 0 && Dv % 8 == 0 && aligned16(p.q) &&
+    using fa::tma_dim_ok;
+    // the tensor-core kernels: head dims up to 128 on the two-tile kernel,
+    // 129..256 on the one-tile (wide) kernel, as for fa_fwd
+    const bool sm100 = (dt == FA_F16 || dt == FA_BF16) && D <= 256 && D % 8 == 0 && Dv % 8 == 0 && aligned16(p.q) &&
                        aligned16(p.k) && aligned16(p.v) && tma_dim_ok(qst, Tq) && tma_dim_ok(qsn, Nq) &&
                        tma_dim_ok(kst, Tk) && tma_dim_ok(ksn, Nk) && tma_dim_ok(vst, Tk) && tma_dim_ok(vsn, Nk);
 
@@ -196,7 +190,11 @@ extern "C" fa_status fa_fwd_varlen_static(
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     unsigned char* dev = static_cast<unsigned char*>(scratch);
 
-    size_t bytes = kCuOffset + kCuBytes;
+    // What this call reads, and nothing more: the ticket counter (zero), the
+    // offsets of its nSeq sequences and, for the tensor-core kernels, its
+    // work table.
+    const size_t tab_off = table_offset(nSeq);
+    size_t bytes = kCuOffset + 2 * (nSeq + 1) * sizeof(int64_t);
     {
         std::lock_guard<std::mutex> lock(g_stage_mutex);
         std::memset(g_host_stage, 0, kCuOffset);  // ticket counter = 0
@@ -208,22 +206,13 @@ extern "C" fa_status fa_fwd_varlen_static(
             cu[nSeq + 2 + b] = actualSeqKvLen[b];
         }
         if (sm100) {
-            int64_t count = 0;
-            for (int64_t b = 0; b < nSeq; ++b) {
-                const int64_t ql = cu[b + 1] - cu[b], kl = cu[nSeq + 2 + b] - cu[nSeq + 1 + b];
-                for (int64_t qb = 0; qb * 256 < ql; ++qb) {
-                    g_cost_stage[count++] = {blocks_for_tile(qb * 256, ql, kl, pre_c, next_c) +
-                                                 blocks_for_tile(qb * 256 + 128, ql, kl, pre_c, next_c),
-                                             make_int4((int)b, (int)qb, (int)ql, (int)kl)};
-                }
-            }
-            std::sort(g_cost_stage, g_cost_stage + count,
-                      [](const CostEntry& a, const CostEntry& c) { return a.cost > c.cost; });
-            int4* table = reinterpret_cast<int4*>(g_host_stage + kTableOffset);
-            for (int64_t e = 0; e < count; ++e) table[e] = g_cost_stage[e].e;
+            const int64_t count = fa::varlen_table_len(cu, nSeq);
+            std::memset(g_host_stage + bytes, 0, tab_off - bytes);  // the alignment gap
+            fa::build_varlen_table(cu, cu + nSeq + 1, nSeq, pre_c, next_c, g_sort_stage,
+                                   reinterpret_cast<int4*>(g_host_stage + tab_off));
             p.table_len = (int32_t)count;
             p.n_items = p.table_len * p.Nq;
-            bytes = kTableOffset + count * sizeof(int4);
+            bytes = tab_off + count * sizeof(int4);
         }
         // Pageable source: staged before the call returns (under stream
         // capture the graph carries the bytes), so the staging buffer may be
@@ -234,7 +223,7 @@ extern "C" fa_status fa_fwd_varlen_static(
     p.cu_kv = p.cu_q + (nSeq + 1);
     cudaError_t err;
     if (sm100) {
-        p.table = reinterpret_cast<const int4*>(dev + kTableOffset);
+        p.table = reinterpret_cast<const int4*>(dev + tab_off);
         int device = 0, sms = 0;
         if (cudaGetDevice(&device) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)

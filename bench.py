@@ -381,33 +381,11 @@ def cpu_threads():
         return os.cpu_count()
 
 
-def run_reference(args, rank):
-    if rank != 0:
-        return
-    w = build(args.workload)
-    for _ in range(args.warmup):
-        time_oracle(w, 0.0, max_heads=1)
-    flops = secs = 0.0
-    heads = 0
-    for _ in range(args.steps):
-        f, s, h = time_oracle(w, 0.0, max_heads=1)
-        flops, secs, heads = flops + f, secs + s, heads + h
-    value = flops / secs / 1e12
-    line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_desc(w),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                         "sample": f"one whole (batch, head) of the workload per step, {heads} heads"},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line), flush=True)
-
-
-def main():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="GPUs (ranks) on this node: under torchrun WORLD_SIZE ranks are already running; "
+                         "without it this script starts one process per GPU itself")
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", type=int, default=2)
@@ -425,33 +403,163 @@ def main():
                     help="TND workload: comma-separated sequence lengths instead of the seeded ones")
     ap.add_argument("--rope", type=int, default=0,
                     help="bf16 workloads: add queryRope/keyRope of this head dim (N(0,1), seeded)")
-    args = ap.parse_args()
+    args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
+    return args
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
-        run_reference(args, rank)
-        return
 
-    import attention_forward_20_b200 as fa
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+def rank_env():
+    """(rank, world size, local rank) from the launcher's environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
 
-    # each rank: its own shard (seed offset by rank) of the workload's batch
+
+def free_port():
+    import socket
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        return sock.getsockname()[1]
+
+
+def spawn_ranks(n, argv, script=None, timeout_s=3600.0):
+    """One process per rank, as torchrun would start them: each runs `script`
+    (this file) with RANK, LOCAL_RANK = rank, WORLD_SIZE = n and a rendezvous
+    on 127.0.0.1 in its environment.  If a rank fails the others are stopped.
+    Returns 0 when every rank exits 0, else the first failing exit code."""
+    import signal
+    import subprocess
+    port = free_port()
+    procs = []
+    for r in range(n):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE=str(n), MASTER_ADDR="127.0.0.1",
+                   MASTER_PORT=str(port))
+        procs.append(subprocess.Popen([sys.executable, script or os.path.abspath(__file__)] + list(argv), env=env,
+                                      start_new_session=True))
+    deadline = time.monotonic() + timeout_s
+    rc = 0
+    while True:
+        codes = [p.poll() for p in procs]
+        failed = [c for c in codes if c not in (None, 0)]
+        if failed or time.monotonic() > deadline:
+            rc = failed[0] if failed else 124
+            for p in procs:
+                if p.poll() is None:
+                    os.killpg(p.pid, signal.SIGTERM)
+            for p in procs:
+                try:
+                    p.wait(timeout=30)
+                except subprocess.TimeoutExpired:
+                    os.killpg(p.pid, signal.SIGKILL)
+                    p.wait()
+            return rc
+        if all(c == 0 for c in codes):
+            return 0
+        time.sleep(0.05)
+
+
+def init_dist(world, backend, device=None):
+    """The process group of a multi-rank run (None for one rank), with a short
+    timeout so that ranks waiting on a failed peer end with an error."""
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    kw = {"device_id": device} if device is not None else {}
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    return dist
+
+
+def prepare_workload(args, rank):
+    """This rank's workload: the configured one, with the flags' variations
+    applied, and its inputs redrawn per rank (rank 0 keeps the workload's own)."""
     w = build(args.workload)
     if args.lengths:
         w = with_lengths(w, args.lengths.split(","))
     if args.head_dim:
         w = with_head_dims(w, args.head_dim, args.value_head_dim or args.head_dim)
-    w = shard_workload(w, rank)
+    return shard_workload(w, rank)
+
+
+def workload_flops(w, rope_dim=0):
+    """(tile-counted, exact) FLOPs of one forward over w; with rope the QK
+    contraction is D + Dr long: 2*(D + Dr) + 2*Dv per counted pair."""
     flops_tiles, flops_exact = tile_flops(w)
+    if rope_dim:
+        d, dv = head_dims(w)
+        f = (2.0 * d + 2.0 * dv + 2.0 * rope_dim) / (2.0 * d + 2.0 * dv)
+        flops_tiles, flops_exact = flops_tiles * f, flops_exact * f
+    return flops_tiles, flops_exact
+
+
+def qkvo_bytes(w):
+    """Bytes of Q, K, V read and O written by one forward over w."""
+    d, dv = head_dims(w)
+    out_elems = w.q.numel() // d * dv
+    es = w.q.element_size()
+    return sum(t.numel() * t.element_size() for t in (w.q, w.k, w.v)) + out_elems * es
+
+
+def workload_config(w, world, args):
+    """The `config` object of the JSON line: the same for both arms."""
+    desc = workload_desc(w)
+    flops_tiles, flops_exact = workload_flops(w, args.rope)
+    if args.kv_chunks > 1:
+        desc["kv_chunks"] = f"{args.kv_chunks} key chunks at their kvStartIdx, then fa_lse_merge (sink added there)"
+    if args.rope:
+        desc["rope"] = f"queryRope/keyRope head dim {args.rope} (bf16, N(0,1)): S = scale*(Q K^T + Qr Kr^T)"
+    if args.pse != "slopes" and w.pse_type == 2:
+        desc["pse"] = ("materialised fp16 bias [1,N,S,S], resident" if args.pse == "dense"
+                       else "compressed bias: last 1024 rows [1,N,1024,S], resident")
+    return dict(desc, parallelism=f"dp{world} (independent shards)",
+                l2=f"flushed before every step (256 MiB write); Q/K/V/O {qkvo_bytes(w) / 1e6:.0f} MB",
+                flops_tile_counted=flops_tiles, flops_exact=flops_exact)
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    w = prepare_workload(args, 0)
+    rope = rope_tensors(w, args.rope, seed=9100) if args.rope else None
+    for _ in range(args.warmup):
+        time_oracle(w, 0.0, max_heads=1, rope=rope)
+    flops = secs = 0.0
+    heads = 0
+    for _ in range(args.steps):
+        f, s_, h = time_oracle(w, 0.0, max_heads=1, rope=rope)
+        flops, secs, heads = flops + f, secs + s_, heads + h
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, args.gpus, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"one whole (batch, head) of the workload per step, {heads} heads"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local_rank = rank_env()
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # not started by torchrun: one process per GPU, started here
+        sys.exit(spawn_ranks(args.gpus, sys.argv[1:] if argv is None else argv))
+    if world > 1 and args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+
+    import attention_forward_20_b200 as fa
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = init_dist(world, "nccl", dev)
+
+    # each rank: its own shard (seed offset by rank) of the workload's batch
+    w = prepare_workload(args, rank)
+    flops_tiles, flops_exact = workload_flops(w, args.rope)
     q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
     kw = fa_kwargs(w, dev)
     rope = None
@@ -460,10 +568,6 @@ def main():
             raise SystemExit("--rope needs a bf16 workload (queryRope/keyRope are BFLOAT16 only)")
         rope = rope_tensors(w, args.rope, seed=9100 + rank)
         kw["query_rope"], kw["key_rope"] = rope[0].to(dev), rope[1].to(dev)
-        # S = Q K^T + Qr Kr^T: 2*(D + Dr) + 2*Dv FLOPs per kept pair
-        d, dv = head_dims(w)
-        flops_tiles *= (2.0 * d + 2.0 * dv + 2.0 * args.rope) / (2.0 * d + 2.0 * dv)
-        flops_exact *= (2.0 * d + 2.0 * dv + 2.0 * args.rope) / (2.0 * d + 2.0 * dv)
     bias_bytes = 0
     if args.pse != "slopes" and w.pse_type == 2:
         # the same ALiBi bias, materialised in the query dtype and resident in HBM
@@ -613,7 +717,6 @@ def main():
         return
 
     ms_per_step = kernel_ms / args.steps
-    qkvo_mb = sum(t.numel() * t.element_size() for t in (q, k, v, out)) / 1e6
     value = whole_job_tflops(flops_tiles, world, ms_per_step)
     per_gpu = flops_tiles / (ms_per_step * 1e-3) / 1e12
     peak, peak_src = load_peak()
@@ -621,30 +724,21 @@ def main():
     fl, secs, heads = time_oracle(w, args.cpu_budget, rope=rope)
     st_value, st_secs = time_oracle_single_thread(w, rope=rope)
     cpu_value = fl / secs / 1e12
-    desc = workload_desc(w)
     merge_line = None
     if args.kv_chunks > 1:
-        desc["kv_chunks"] = f"{args.kv_chunks} key chunks at their kvStartIdx, then fa_lse_merge (sink added there)"
         timed = merge_events[-args.steps:]
         merge_ms = sum(a.elapsed_time(b) for a, b in timed) / max(1, len(timed))
         part_bytes = out.numel() * out.element_size() + 2 * smax.numel() * smax.element_size()
         merge_line = hbm_line(0, q, k, v, out, merge_ms, bytes_override=(args.kv_chunks + 1) * part_bytes)
         merge_line["ms"] = merge_ms
-    if rope is not None:
-        desc["rope"] = f"queryRope/keyRope head dim {args.rope} (bf16, N(0,1)): S = scale*(Q K^T + Qr Kr^T)"
-    if args.pse != "slopes" and w.pse_type == 2:
-        desc["pse"] = ("materialised fp16 bias [1,N,S,S], resident" if args.pse == "dense"
-                       else "compressed bias: last 1024 rows [1,N,1024,S], resident")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": dict(desc, parallelism=f"dp{world} (independent shards)",
-                       l2=f"flushed before every step (256 MiB write); Q/K/V/O {qkvo_mb:.0f} MB",
-                       flops_tile_counted=flops_tiles, flops_exact=flops_exact,
-                       pct_of_nominal_2250=100.0 * per_gpu / 2250.0),
+        "config": workload_config(w, world, args),
         "roofline": {"bound": "tensor", "achieved": per_gpu, "peak": peak, "unit": UNIT,
-                     "frac": per_gpu / peak, "traffic": traffic, "peak_source": peak_src},
+                     "frac": per_gpu / peak, "traffic": traffic, "peak_source": peak_src,
+                     "pct_of_nominal_2250": 100.0 * per_gpu / 2250.0},
         **({"hbm": hbm_line(bias_bytes, q, k, v, out, ms_per_step)} if args.pse == "dense" else {}),
         **({"merge": merge_line} if merge_line else {}),
         "cpu_baseline": {"value": cpu_value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",

@@ -269,16 +269,19 @@ FA_API fa_status fa_device_error(uint64_t* detail);
  * static array (about 130 KB: the offsets and up to 6144 work items) is held
  * on every GPU that loads the library until the process exits.
  *
- * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  Every call overwrites the part of the array it reads, so nothing
+ * The first call on a device looks up the array's device address (with that
+ * device current) and keeps it once the lookup succeeds; make that first call
+ * before any stream capture.  Every call overwrites the part of the array it reads, so nothing
  * needs clearing, but calls whose work overlaps on the GPU (other streams,
  * other host threads) race on the shared array.  Under stream capture the
  * offsets and table travel in the graph (copy kernels that carry the bytes in
  * their launch parameters), so each replay writes its own table back into the
  * array first; replays, like calls, must not overlap on the GPU.
- * fp16/bf16 with head dims up to 128 run on the tensor cores, the rest on the
- * CUDA-core kernel.
+ * Each call uploads only what it reads (the ticket counter, its nSeq + 1
+ * offsets per side and its work table).  Kernel choice is fa_fwd's:
+ * fp16/bf16 with head dims that are multiples of 8 up to 256 run on the
+ * tensor cores (the two-tile kernel up to 128, the one-tile kernel above),
+ * fp32 and other head dims on the CUDA-core kernel.
  *
  * Returns FA_SUCCESS, FA_ERR_PARAM_NULLPTR, FA_ERR_PARAM_INVALID,
  * FA_ERR_INNER_NULLPTR or FA_ERR_CUDA. */

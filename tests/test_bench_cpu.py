@@ -1,7 +1,6 @@
 """The bench's host logic on CPU: the FLOP counts it divides by (closed forms
 and brute-force tile counts), the inputs it builds for other head dims and for
 rope, and the reference arm's JSON line."""
-import argparse
 import contextlib
 import io
 import json
@@ -77,7 +76,7 @@ def test_rope_tensors_follow_the_layout():
 
 
 def test_reference_arm_line():
-    args = argparse.Namespace(workload=1, steps=2, warmup=3, gpus=1)
+    args = bench.parse_args(["--workload", "1", "--steps", "2", "--warmup", "3", "--impl", "reference"])
     buf = io.StringIO()
     with contextlib.redirect_stdout(buf):
         bench.run_reference(args, rank=0)

@@ -1,8 +1,12 @@
 """The bench's multi-rank host logic on CPU: two gloo ranks take distinct
 shards, the timing reduction is a max over ranks, and the whole-job value
 counts every rank's units over the slowest rank's time."""
+import contextlib
+import io
+import json
 import os
 import socket
+import time
 
 import torch
 import torch.distributed as dist
@@ -45,3 +49,39 @@ def test_two_gloo_ranks_shard_and_reduce():
     # rank 0 keeps the workload's own inputs
     w = build(2, seq_scale=64)
     assert abs(float(w.q.float().sum()) - float(sums0[0][0])) < 1e-3
+
+
+RANK_SCRIPT = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_bench_rank_cpu.py")
+
+
+def test_spawn_ranks_runs_the_sharded_path_on_two_gloo_ranks(capfd):
+    """bench.py --gpus 2 without torchrun: spawn_ranks starts one process per
+    rank (the environment torchrun would give), each prepares and shards its
+    workload as main() does, the step time is the max over ranks, and rank 0
+    prints a line whose n_gpus is 2 and whose value counts both ranks' work."""
+    argv = ["--gpus", "2", "--workload", "1", "--steps", "2", "--warmup", "3"]
+    assert bench.spawn_ranks(2, argv, script=RANK_SCRIPT, timeout_s=300) == 0
+    lines = [ln for ln in capfd.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1                       # rank 0 alone prints
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2
+    assert line["ms_per_step"] >= 20.0           # the slower rank's time
+    assert abs(line["value"] - 2 * line["flops_per_rank"] / (line["ms_per_step"] * 1e-3) / 1e12) < 1e-12
+    assert line["config"]["parallelism"] == "dp2 (independent shards)"
+    c0, c1 = line["checksums"]
+    assert c0 != c1                              # distinct shards
+    w = build(1)                                 # rank 0 keeps the workload's own inputs
+    assert abs(float(w.q.double().sum()) - c0[0]) < 1e-9
+    # the reference arm reports the same config for the same workload
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.run_reference(bench.parse_args(argv + ["--impl", "reference"]), rank=0)
+    assert json.loads(buf.getvalue().strip().splitlines()[-1])["config"] == line["config"]
+
+
+def test_spawn_ranks_stops_the_others_when_a_rank_fails(monkeypatch):
+    monkeypatch.setenv("FAIL_RANK", "1")
+    argv = ["--gpus", "2", "--workload", "1"]
+    t0 = time.monotonic()
+    assert bench.spawn_ranks(2, argv, script=RANK_SCRIPT, timeout_s=300) == 3
+    assert time.monotonic() - t0 < 120           # rank 0 did not wait for its peer's timeout

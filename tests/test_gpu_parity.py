@@ -89,6 +89,45 @@ def test_band_alibi_two_sided():
     compare_full(w)
 
 
+def _per_batch_slopes(n_batch, n_heads):
+    """fp32 [B, N] ALiBi slopes, different along both axes and not symmetric."""
+    b = torch.arange(n_batch, dtype=torch.float64)[:, None]
+    n = torch.arange(n_heads, dtype=torch.float64)[None, :]
+    return (2.0 ** -(n + 1) * (1 + 0.37 * b) + 0.05 * n * b).to(torch.float32)
+
+
+@pytest.mark.parametrize("case", ["two_tile_bsnd_d64", "two_tile_tnd_d128", "wide_bnsd_d256", "cuda_core_f32"])
+def test_alibi_per_batch_slopes(case):
+    """Slope-only pse of shape [B, N] (aclnnFlashAttentionVarLenScoreV5,
+    realShiftOptional notes): batch row (TND: sequence) b of head n uses
+    slope[b, n], on each of the three kernels."""
+    if case == "two_tile_bsnd_d64":
+        w = W("BSND", "f16", (3, 300, 3, 64), 3, 460, pre_tokens=150, next_tokens=0)
+        kernel = "sm100_tcgen05"
+    elif case == "two_tile_tnd_d128":
+        lens = [23, 400, 170]
+        cum = cumulative(lens, False)
+        w = W("TND", "bf16", (sum(lens), 2, 128), 2, 470, actual_seq_q=cum, actual_seq_kv=list(cum),
+              pre_tokens=200, next_tokens=30)
+        kernel = "sm100_tcgen05"
+    elif case == "wide_bnsd_d256":
+        w = W("BNSD", "bf16", (2, 2, 260, 256), 2, 480, pre_tokens=100, next_tokens=0)
+        kernel = "sm100_tcgen05"
+    else:
+        w = W("BNSD", "f32", (2, 3, 150, 64), 3, 490, pre_tokens=60, next_tokens=5)
+        kernel = "simt"
+    n_batch = len(w.actual_seq_q) if w.layout == "TND" else w.q.shape[0]
+    w.pse, w.pse_type = _per_batch_slopes(n_batch, w.head_num), 2
+    assert kernel in plan_text(w)
+    compare_full(w)
+    # every batch row given row 0's slopes: the same bits as the [N] form
+    rows_equal = w.pse[:1].expand(n_batch, -1).contiguous()
+    a = run_gpu(w, real_shift=rows_equal.cuda())
+    b = run_gpu(w, real_shift=w.pse[0].contiguous().cuda())
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 def test_dense_pse_tensor(dtype):
     s = 260
@@ -343,13 +382,51 @@ def test_outputs_fully_written():
 # the five workloads at full size, as the bench launches them: sampled rows
 # ---------------------------------------------------------------------------
 
+def _split_item_rows(w, text):
+    """(b, n, i) rows of every split work item of a dense-layout launch: the
+    first, a middle and the last row of each of its two 128-row tiles.
+
+    Work item u of the dense layouts is (head bn, query block qb) with the
+    heads in groups of `head_group`; inside a group the query blocks run from
+    the last to the first, heads fastest.  The split items are the last
+    `split_items` of that order."""
+    n_split = int(text.split("split_items=")[1].split()[0])
+    if n_split == 0:
+        return []
+    sq = {"BNSD": w.q.shape[2], "BSND": w.q.shape[1], "BSH": w.q.shape[1], "SBH": w.q.shape[0]}[w.layout]
+    bsz = w.q.shape[1] if w.layout == "SBH" else w.q.shape[0]
+    d = w.q.shape[-1] if w.layout not in ("BSH", "SBH") else w.q.shape[-1] // w.head_num
+    hg = 4 if d > 128 else 16
+    n_qb = (sq + 255) // 256
+    bn_total = bsz * w.head_num
+    n_items = n_qb * bn_total
+    assert f"items={n_items} " in text
+    rows = []
+    for u in range(n_items - n_split, n_items):
+        g, within = divmod(u, hg * n_qb)
+        g_heads = min(hg, bn_total - g * hg)
+        level, h = divmod(within, g_heads)
+        b, n = divmod(g * hg + h, w.head_num)
+        qb = n_qb - 1 - level
+        for r in (0, 63, 127, 128, 200, 255):
+            if qb * 256 + r < sq:
+                rows.append((b, n, qb * 256 + r))
+    return rows
+
+
 @pytest.mark.parametrize("number", [1, 2, 3, 4, 5])
 def test_full_size_workloads_sampled(number):
     w = build(number)
     res = run_gpu(w)
     for t in res:
         assert not torch.isnan(t).any()
-    compare_rows(w, res, sample_rows(w, 24, seed=number))
+    rows = sample_rows(w, 24, seed=number)
+    if w.layout != "TND" and w.dtype != "f32":
+        split_rows = _split_item_rows(w, plan_text(w))
+        if number == 2:  # the headline launch splits its short last wave
+            assert len(split_rows) >= 2 * 6, "expected split items in the headline launch"
+        rows += split_rows
+    compare_rows(w, res, rows)
 
 
 # ---------------------------------------------------------------------------

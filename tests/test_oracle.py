@@ -239,6 +239,52 @@ def test_alibi_geometric_series():
             np.testing.assert_allclose(res["softmax_sum"][0, n, i], l_exact, rtol=1e-13)
 
 
+def per_batch_slopes(n_batch, n_heads):
+    """fp32 [B, N] ALiBi slopes that differ along both axes and are not
+    symmetric: slope[b, n] = 2^(-(n+1)) * (1 + 0.37 b) + 0.05 n b."""
+    b = np.arange(n_batch, dtype=np.float64)[:, None]
+    n = np.arange(n_heads, dtype=np.float64)[None, :]
+    return (2.0 ** -(n + 1) * (1 + 0.37 * b) + 0.05 * n * b).astype(np.float32)
+
+
+@pytest.mark.parametrize("layout", ["BSND", "TND"])
+def test_alibi_geometric_series_per_batch_slopes(layout):
+    """The [B, N] slope form (aclnnFlashAttentionVarLenScoreV5, realShiftOptional
+    notes: a slope-only pse of shape [B, N] or [N]): batch row b, head n use
+    slope[b, n].  Q = 0, causal band of width pre: l = (1 - r^(K+1))/(1 - r)
+    with r = e^-slope[b, n] and K = min(i, pre), as for [N] slopes, but with a
+    different r for every (b, n); for TND, b is the sequence."""
+    n_batch, n_heads, pre = 3, 3, 9
+    slopes = per_batch_slopes(n_batch, n_heads).astype(np.float64)
+    assert not np.allclose(slopes, slopes.T)
+    if layout == "BSND":
+        lens = [40] * n_batch
+        q = np.zeros((n_batch, 40, n_heads, 8))
+        k, v = rand((n_batch, 40, n_heads, 8), 65), rand((n_batch, 40, n_heads, 8), 66)
+        res = ref.forward(q, k, v, layout="BSND", head_num=n_heads, scale=1.0,
+                          pse=slopes, pse_type=2, pre_tokens=pre, next_tokens=0)
+        lsum = lambda b, n, i: res["softmax_sum"][b, n, i]  # noqa: E731
+        lmax = lambda b, n, i: res["softmax_max"][b, n, i]  # noqa: E731
+    else:
+        lens = [23, 40, 17]
+        t = sum(lens)
+        q = np.zeros((t, n_heads, 8))
+        k, v = rand((t, n_heads, 8), 67), rand((t, n_heads, 8), 68)
+        cu = cumulative(lens, False)
+        res = ref.forward(q, k, v, layout="TND", head_num=n_heads, scale=1.0, pse=slopes, pse_type=2,
+                          pre_tokens=pre, next_tokens=0, actual_seq_q=cu, actual_seq_kv=cu)
+        starts = [0] + cu[:-1]
+        lsum = lambda b, n, i: res["softmax_sum"][n, starts[b] + i]  # noqa: E731
+        lmax = lambda b, n, i: res["softmax_max"][n, starts[b] + i]  # noqa: E731
+    for b in range(n_batch):
+        for n in range(n_heads):
+            r = math.exp(-slopes[b, n])
+            for i in range(lens[b]):
+                kk = min(i, pre)
+                assert np.all(lmax(b, n, i) == 0.0)
+                np.testing.assert_allclose(lsum(b, n, i), (1 - r ** (kk + 1)) / (1 - r), rtol=1e-13)
+
+
 def test_alibi_symmetric_band():
     """Q = 0, ALiBi slope s, band [i - pre, i + next]: the kept weights are
     r^|i-j|, so l = sum over the two one-sided geometric series

@@ -36,6 +36,10 @@ MUTATIONS = [
     ("mask polarity inverted", "keep &= ~np.asarray(excluded[r0:r1], dtype=bool)",
      "keep &= np.asarray(excluded[r0:r1], dtype=bool)"),
     ("ALiBi sign flipped", "return -slope * np.abs(", "return slope * np.abs("),
+    ("ALiBi [B, N] slopes indexed [n, b]", "slope = pse[b, n] if pse.ndim == 2 else pse[n]",
+     "slope = pse[n, b] if pse.ndim == 2 else pse[n]"),
+    ("ALiBi [B, N] slopes ignore the batch row", "slope = pse[b, n] if pse.ndim == 2 else pse[n]",
+     "slope = pse[0, n] if pse.ndim == 2 else pse[n]"),
     ("ALiBi without abs", "np.abs(np.asarray(rows, dtype=np.float64)[:, None] - j[None, :])",
      "(np.asarray(rows, dtype=np.float64)[:, None] - j[None, :])"),
     ("BSH split order", "x.reshape(b, s, h // head_dim, head_dim).transpose(0, 2, 1, 3)",
@@ -88,6 +92,8 @@ def _run_pins():
     for args in [(40, 40, INT64_MAX, 0), (40, 40, 7, 0), (33, 50, 4, 9), (50, 20, 0, 0), (25, 25, 3, -2)]:
         pins.test_zero_query_band_counts(*args)
     pins.test_alibi_geometric_series()
+    for layout in ("BSND", "TND"):
+        pins.test_alibi_geometric_series_per_batch_slopes(layout)
     pins.test_alibi_symmetric_band()
     pins.test_empty_rows()
     pins.test_identity_value_exposes_probability_rows()
