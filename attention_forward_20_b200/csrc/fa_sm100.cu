@@ -54,13 +54,41 @@ constexpr int kTileM = 128;     // query rows per tile (one TMEM lane each)
 constexpr int kTileN = 128;     // keys per block
 constexpr int kQBlock = 256;    // query rows per work item (two tiles)
 constexpr int kThreads = 384;   // three warpgroups
-constexpr uint32_t kSoftmaxRegs = 216;  // per thread, softmax warpgroups (setmaxnreg)
-constexpr uint32_t kOtherRegs = 72;     // per thread, producer/MMA warpgroup
+// Per-thread registers after setmaxnreg: softmax warpgroups / producer-MMA
+// warpgroup.  The rope kernels' producer and MMA warps keep more state.
+template <bool kRope>
+constexpr uint32_t kSoftmaxRegs = kRope ? 216 : 224;
+template <bool kRope>
+constexpr uint32_t kOtherRegs = kRope ? 72 : 56;
+// setmaxnreg hands out what the launch reserved: 384 threads x 168 registers
+// (the allocation unit is 8 registers per thread; 176 x 384 exceeds 64K)
+static_assert(2 * 128 * kSoftmaxRegs<false> + 128 * kOtherRegs<false> <= (65536 / kThreads) / 8 * 8 * kThreads &&
+                  2 * 128 * kSoftmaxRegs<true> + 128 * kOtherRegs<true> <= (65536 / kThreads) / 8 * 8 * kThreads,
+              "register split exceeds the launch's reservation");
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kRescaleThreshold = 8.0f;
+
+// Column pairs, of every 8 in a score row, whose exponentials run on the FMA
+// pipe (exp2_fma2) instead of MUFU, by padded head dim: MUFU bounds the
+// softmax at every head dim (16 exponentials per clock per SM), the FMA pipe
+// has room beside it.
+#ifndef FA_POLY_PAIRS_64
+#define FA_POLY_PAIRS_64 0
+#endif
+#ifndef FA_POLY_PAIRS_128
+#define FA_POLY_PAIRS_128 0
+#endif
+#ifndef FA_POLY_PAIRS_256
+#define FA_POLY_PAIRS_256 0
+#endif
+template <int D>
+constexpr int kPolyPairs = D <= 64 ? FA_POLY_PAIRS_64 : (D <= 128 ? FA_POLY_PAIRS_128 : FA_POLY_PAIRS_256);
+static_assert(kPolyPairs<64> >= 0 && kPolyPairs<64> <= 8 && kPolyPairs<128> >= 0 && kPolyPairs<128> <= 8 &&
+                  kPolyPairs<256> >= 0 && kPolyPairs<256> <= 8,
+              "poly pairs per 8");
 constexpr int kSched = 4;            // ticket slots between the TMA warp and the other warps
 constexpr int kTicketEnd = -1;       // no work left
 constexpr int kTicketAbort = -2;     // a bounded wait gave up
@@ -93,6 +121,7 @@ static_assert(Cfg<64, true>::kSmemBytes + 1024 <= 227 * 1024, "rope tiles exceed
 
 struct Barriers {
     uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2];
+    uint64_t p_half[2];    // two-tile kernel: the first 64 keys' half of P_t is in TMEM
     uint64_t kv_full[8], kv_empty[8];
     uint64_t kr_empty[2];  // keyRope slots (the K load's kv_full also covers its keyRope chunk)
     uint64_t pv_done;      // wide kernel: one completion per key block's P·V
@@ -391,6 +420,10 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* s
         ++kv_use;
         return r;
     };
+    // One elected lane (elect.sync: the same lane every time in a converged
+    // warp) issues every MMA and commit, so its commits track its MMAs; the
+    // descriptors of the fixed shared-memory buffers are computed once, slot
+    // k of the ring being kTileBytes further.
     auto commit = [&](uint64_t* bar) {
         if (elect_one()) tc_commit(bar);
         __syncwarp();
@@ -398,12 +431,17 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* s
     // S_t = Q_t · K^T: D/16 MMAs of K = 16; both operands K-major, 128-byte
     // swizzled, 8-row groups 1024 bytes apart, 64-column chunks one tile-chunk apart.
     // S_t = Q_t · K^T over D/16 K-steps, O_t (+)= P_t · V over 8 K-steps:
-    // each group is one asm block issued by one elected lane.
+    // each group is one asm block issued by one lane.
     // With rope, 4 more K-steps over the queryRope / keyRope chunks accumulate
     // into the same S.
+    constexpr uint64_t kSlotDesc = C::kTileBytes >> 4;  // descriptor start-address units of 16 bytes
+    const uint64_t qdesc[2] = {sdesc_sw128(smem_u32(sQ), 1024, 16),
+                               sdesc_sw128(smem_u32(sQ + C::kQTileBytes), 1024, 16)};
+    const uint64_t kdesc0 = sdesc_sw128(smem_u32(sKV), 1024, 16);
+    const uint64_t vdesc0 = sdesc_sw128(smem_u32(sKV), 1024, C::kChunkBytes);
     auto issue_qk = [&](int t, int slot, uint32_t rs) {
-        const uint64_t qd = sdesc_sw128(smem_u32(sQ + t * C::kQTileBytes), 1024, 16);
-        const uint64_t kd = sdesc_sw128(smem_u32(sKV + slot * C::kTileBytes), 1024, 16);
+        const uint64_t qd = t ? qdesc[1] : qdesc[0];
+        const uint64_t kd = kdesc0 + static_cast<uint64_t>(slot) * kSlotDesc;
         if (elect_one()) {
             if constexpr (D == 128)
                 mma_ss_k128(tmem + t * kTileN, qd, kd, idesc_qk, 0u);
@@ -417,9 +455,12 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* s
         }
         __syncwarp();
     };
-    auto issue_pv = [&](int t, int slot, bool accumulate) {
-        const uint64_t vd = sdesc_sw128(smem_u32(sKV + slot * C::kTileBytes), 1024, C::kChunkBytes);
-        if (elect_one()) mma_ts_k128(tmem + kOCol + t * D, tmem + t * kTileN, vd, idesc_pv, accumulate ? 1u : 0u);
+    // O_t (+)= P_t · V over the block's keys 64h .. 64h+63: P columns 32h..,
+    // V rows from 64h (4 K-steps of 16 keys, 2048 bytes each)
+    auto issue_pv_half = [&](int t, int slot, int h, bool accumulate) {
+        const uint64_t vd = vdesc0 + static_cast<uint64_t>(slot) * kSlotDesc + static_cast<uint64_t>(h) * (4 * 2048 / 16);
+        if (elect_one())
+            mma_ts_k64(tmem + kOCol + t * D, tmem + t * kTileN + 32 * h, vd, idesc_pv, accumulate ? 1u : 0u);
         __syncwarp();
     };
 
@@ -458,10 +499,15 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* s
             rs = kr_use % 2;
             for (int t = 0; t < 2; ++t) {
                 if (tr[t].has(jb)) {
+                    // the first half of P·V as soon as the softmax has stored
+                    // that half of P, the second after the whole of P
+                    if (!warp_wait(&bars.p_half[t], p_cnt[t] & 1, abort, kSitePFull)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv_half(t, sv, 0, jb != tr[t].lo);
                     if (!warp_wait(&bars.p_full[t], p_cnt[t] & 1, abort, kSitePFull)) { ok = false; break; }
                     ++p_cnt[t];
                     tc_fence_after();
-                    issue_pv(t, sv, jb != tr[t].lo);
+                    issue_pv_half(t, sv, 1, true);
                     if (jb == tr[t].hi) commit(&bars.o_full[t]);
                 }
                 if (has_next && tr[t].has(jb + 1)) {
@@ -986,30 +1032,17 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
             m_run = m_new;
             const float shift = (m_used == -CUDART_INF_F) ? 0.f : m_used;
 
-            // p = 2^(x - shift), two columns per packed FMA / ADD / convert
+            // p = 2^(x - shift), two columns per packed FMA / ADD / convert;
+            // kPolyPairs of every 8 column pairs take the FMA-pipe exponential
+            // (spread over the 8), the others MUFU's ex2
             float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
             const float mult = kBias ? 1.f : sl2;
             const float nshift = row_off - shift;
-            uint32_t pk[64];
-#pragma unroll
-            for (int c = 0; c < kTileN; c += 4) {
-                float x0, x1, x2, x3;
-                fma2(x0, x1, s[c], s[c + 1], mult, mult, nshift, nshift);
-                fma2(x2, x3, s[c + 2], s[c + 3], mult, mult, nshift, nshift);
-                const float e0 = ex2(x0), e1 = ex2(x1), e2 = ex2(x2), e3 = ex2(x3);
-                add2(l0, l1, e0, e1);
-                add2(l2, l3, e2, e3);
-                pk[c / 2] = pack2<T>(e0, e1);
-                pk[c / 2 + 1] = pack2<T>(e2, e3);
-            }
-            l += (l0 + l1) + (l2 + l3);
-            tmem_st_x64(tS, pk);
-            if (jb > tr.lo && __any_sync(0xffffffffu, need)) {
-                // Rescale O_t by alpha before this block's P·V is issued.  Two
-                // tiles: O_t is stable, the commit behind this block's S_t covered
-                // the last P·V.  Wide: wait for the previous block's P·V.
-                if (kWide && !warp_wait(&bars.pv_done, (g_blk - 1) & 1, abort, kSiteOFull)) { ok = false; break; }
-                if (kWide) tc_fence_after();
+            // Rescale O_t by alpha before this block's P·V reaches it.  Two
+            // tiles: O_t is stable, the commit behind this block's S_t covered
+            // the last P·V.  Wide: wait for the previous block's P·V first.
+            const bool rescale = jb > tr.lo && __any_sync(0xffffffffu, need);
+            auto rescale_o = [&]() {
 #pragma unroll
                 for (int cc = 0; cc < D; cc += 32) {
                     if (cc >= p.Dv) break;
@@ -1019,6 +1052,53 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                     tmem_st_x32(tO + cc, o);
                 }
+            };
+            // P goes to TMEM in two halves of 64 columns (only one half's
+            // packed values live at a time).  Two tiles: p_half releases the
+            // first half's P·V (over keys 0..63) while the second half of
+            // the exponentials runs.
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c4 = 0; c4 < 64; c4 += 4) {
+                    const int c = 64 * h + c4;
+                    float x0, x1, x2, x3, e0, e1, e2, e3;
+                    fma2(x0, x1, s[c], s[c + 1], mult, mult, nshift, nshift);
+                    fma2(x2, x3, s[c + 2], s[c + 3], mult, mult, nshift, nshift);
+                    constexpr int P = kPolyPairs<D>;
+                    if (((c / 2) * P) % 8 < P) {
+                        exp2_fma2(x0, x1, e0, e1);
+                    } else {
+                        e0 = ex2(x0);
+                        e1 = ex2(x1);
+                    }
+                    if (((c / 2 + 1) * P) % 8 < P) {
+                        exp2_fma2(x2, x3, e2, e3);
+                    } else {
+                        e2 = ex2(x2);
+                        e3 = ex2(x3);
+                    }
+                    add2(l0, l1, e0, e1);
+                    add2(l2, l3, e2, e3);
+                    pk[c4 / 2] = pack2<T>(e0, e1);
+                    pk[c4 / 2 + 1] = pack2<T>(e2, e3);
+                }
+                tmem_st_x32(tS + 32 * h, pk);
+                if constexpr (!kWide) {
+                    if (h == 0) {
+                        if (rescale) rescale_o();
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(&bars.p_half[sb]);
+                    }
+                }
+            }
+            l += (l0 + l1) + (l2 + l3);
+            if (kWide && rescale) {
+                if (!warp_wait(&bars.pv_done, (g_blk - 1) & 1, abort, kSiteOFull)) { ok = false; break; }
+                tc_fence_after();
+                rescale_o();
             }
             tmem_wait_st();
             tc_fence_before();
@@ -1170,6 +1250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars.q_empty[t], 1);
             mbar_init(&bars.s_full[t], 1);
             mbar_init(&bars.p_full[t], kTileM);
+            mbar_init(&bars.p_half[t], kTileM);
             mbar_init(&bars.o_full[t], 1);
         }
         for (int s = 0; s < C::kStages; ++s) {
@@ -1205,10 +1286,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = tmem_base;
 
     if (warp < 8) {
-        setmaxnreg_inc<kSoftmaxRegs>();
+        setmaxnreg_inc<kSoftmaxRegs<kRope>>();
         run_softmax<T, D, kBias>(p, bars, slots, tmem, &abort_flag, warp >> 2);
     } else {
-        setmaxnreg_dec<kOtherRegs>();
+        setmaxnreg_dec<kOtherRegs<kRope>>();
         if (warp == kLoadWarp)
             run_producer<D, kRope>(p, &tmap_q, &tmap_k, &tmap_v, &tmap_qr, &tmap_kr, sQ, sKV, sKr, bars, slots,
                                    &abort_flag);
@@ -1318,7 +1399,7 @@ cudaError_t launch_t(const FaParams& p, const TmaSet& maps, int num_sms, cudaStr
     cudaFuncAttributes attr{};
     e = cudaFuncGetAttributes(&attr, kern);
     if (e != cudaSuccess) return e;
-    if (static_cast<uint64_t>(attr.numRegs) * kThreads < 2ull * 128 * kSoftmaxRegs + 128ull * kOtherRegs)
+    if (static_cast<uint64_t>(attr.numRegs) * kThreads < 2ull * 128 * kSoftmaxRegs<kRope> + 128ull * kOtherRegs<kRope>)
         return cudaErrorLaunchOutOfResources;
     (void)num_sms;
     if (p.grid <= 0) return cudaSuccess;

@@ -251,6 +251,26 @@ __device__ __forceinline__ void mma_ts_k128(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
+// O (+)= P·V over 4 K-steps of 16 keys (half of a 128-key block): P in TMEM
+// (8 columns per step), V an MN-major 128-byte-swizzled smem tile (step k
+// starts k*2048 bytes in).  The first step accumulates iff `accumulate`.
+__device__ __forceinline__ void mma_ts_k64(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .b64 db;\n\t.reg .b32 ta;\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "add.s32 ta, %1, 8;\n\tadd.s64 db, %2, 128;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+        "add.s32 ta, %1, 16;\n\tadd.s64 db, %2, 256;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+        "add.s32 ta, %1, 24;\n\tadd.s64 db, %2, 384;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+        "}\n"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor for a tile written by TMA with 128-byte
 // swizzling: 8-row x 128-byte swizzle atoms, `sbo` bytes between 8-row groups
 // along M/N (K-major) or along K (MN-major), `lbo` bytes between 64-element
@@ -459,6 +479,55 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// (d0, d1) = (a0 - b0, a1 - b1), round to nearest, one packed instruction.
+__device__ __forceinline__ void sub2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
+        "mov.b64 pa, {%2, %3};\n\t"
+        "mov.b64 pb, {%4, %5};\n\t"
+        "sub.rn.f32x2 pd, pa, pb;\n\t"
+        "mov.b64 {%0, %1}, pd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// (d0, d1) = (a0 + b, a1 + b) rounded toward -inf, one packed instruction.
+__device__ __forceinline__ void add2_rm(float& d0, float& d1, float a0, float a1, float b) {
+    asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
+        "mov.b64 pa, {%2, %3};\n\t"
+        "mov.b64 pb, {%4, %4};\n\t"
+        "add.rm.f32x2 pd, pa, pb;\n\t"
+        "mov.b64 {%0, %1}, pd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b));
+}
+
+// 2^x for two values on the FMA pipe instead of MUFU (so that a share of a
+// row's exponentials can run beside the MUFU ones).  Cody-Waite style split
+// x = j + f, j = floor(x), f in [0, 1): adding 1.5 * 2^23 rounded toward -inf
+// leaves j in the low mantissa bits of t (exact for |x| < 2^22), f = x -
+// (t - 1.5 * 2^23) is exact, 2^f comes from a degree-3 polynomial with
+// p(0) = 1 (coefficients: the minimax relative-error fit of 2^f on [0, 1]
+// that exp2_poly_fit.py computes; largest relative error 8.6e-5), and j is
+// added to the exponent field (t << 23 is j << 23 modulo 2^32).  x is first
+// clamped to -127: any x <= -127 (also -inf) gives j = -127, f = 0, p = 1
+// and exactly +0.0; results below 2^-126 are not accurate (they only ever
+// meet sums of at least 1).
+__device__ __forceinline__ void exp2_fma2(float x0, float x1, float& y0, float& y1) {
+    constexpr float kShifter = 12582912.0f;  // 1.5 * 2^23
+    constexpr float c1 = 0.69511676f, c2 = 0.227645f, c3 = 0.07706704f;
+    x0 = fmaxf(x0, -127.0f);
+    x1 = fmaxf(x1, -127.0f);
+    float t0, t1, j0, j1, f0, f1, p0, p1;
+    add2_rm(t0, t1, x0, x1, kShifter);
+    sub2(j0, j1, t0, t1, kShifter, kShifter);
+    sub2(f0, f1, x0, x1, j0, j1);
+    fma2(p0, p1, f0, f1, c3, c3, c2, c2);
+    fma2(p0, p1, p0, p1, f0, f1, c1, c1);
+    fma2(p0, p1, p0, p1, f0, f1, 1.0f, 1.0f);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 }  // namespace ptx

@@ -403,6 +403,9 @@ def parse_args(argv=None):
                     help="TND workload: comma-separated sequence lengths instead of the seeded ones")
     ap.add_argument("--rope", type=int, default=0,
                     help="bf16 workloads: add queryRope/keyRope of this head dim (N(0,1), seeded)")
+    ap.add_argument("--seq-scale", type=int, default=1,
+                    help="divide the workload's sequence lengths (and the band's preTokens) by this factor: "
+                         "a smaller case of the same structure, for profiler captures")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     return args
@@ -472,7 +475,9 @@ def init_dist(world, backend, device=None):
 def prepare_workload(args, rank):
     """This rank's workload: the configured one, with the flags' variations
     applied, and its inputs redrawn per rank (rank 0 keeps the workload's own)."""
-    w = build(args.workload)
+    w = build(args.workload, seq_scale=args.seq_scale)
+    if args.seq_scale > 1:
+        w.name = f"{w.name}_seq_div{args.seq_scale}"
     if args.lengths:
         w = with_lengths(w, args.lengths.split(","))
     if args.head_dim:

@@ -11,8 +11,9 @@ Roles, in the order `run_producer`, `run_mma` and `run_softmax` use them:
             tile that has j: P(t, j), P·V, o_full[t] on its last block; for
             each tile that has j+1: S(t, j+1) (after that tile's P·V, since P
             aliases S in TMEM), q_empty[t] after its last S;
-  softmax t: per item, for each block of its range: S then P; o_full[t]
-            before the epilogue when it had blocks.
+  softmax t: per item, for each block of its range: S, then (after any O
+            rescale) the first half of P (p_half), then the rest (p_full);
+            o_full[t] before the epilogue when it had blocks.
 Checks: random interleavings finish; no wait passes before its phase; ring
 slots hold what the MMA expects; every S reads the Q tile of its own item;
 S(t, j+1) is issued after P·V(t, j); a tile's first P·V of an item (which
@@ -152,11 +153,18 @@ def run(items, stages, rope, seed):
                 sk2 = (yield from take(("K", j + 1))) if nxt else None
                 for t in range(2):
                     if has(tr[t], j):
-                        yield ("wait", f"p_full{t}", p_cnt[t] & 1, p_cnt[t])
-                        p_cnt[t] += 1
+                        # P·V in two halves: keys 0..63 once the softmax has
+                        # stored that half of P, keys 64..127 after the rest
+                        yield ("wait", f"p_half{t}", p_cnt[t] & 1, p_cnt[t])
+                        assert ("Phalf", t, j) in log, ("P·V over a half of P not yet stored", t, j)
                         if j == tr[t]["lo"]:
                             assert epilogues[t] == items_started[t], ("O overwritten before the epilogue", t)
                             items_started[t] += 1
+                        assert ring.get(sv) == ("V", j), ("P·V reads a slot that no longer holds V", j)
+                        log.append(("PVlo", t, j))
+                        yield ("wait", f"p_full{t}", p_cnt[t] & 1, p_cnt[t])
+                        p_cnt[t] += 1
+                        assert ("P", t, j) in log, ("P·V over P not yet stored", t, j)
                         assert ring.get(sv) == ("V", j), ("P·V reads a slot that no longer holds V", j)
                         log.append(("PV", t, j))
                         if j == tr[t]["hi"]:
@@ -182,6 +190,13 @@ def run(items, stages, rope, seed):
                 yield ("wait", f"s_full{t}", s_cnt & 1, s_cnt)
                 s_cnt += 1
                 assert ("S", t, j) in log, ("S read before it was computed", t, j)
+                if j > r["lo"]:
+                    # an O rescale happens here, before the first half's arrival
+                    assert ("PV", t, j - 1) in log, ("O rescaled before the last P·V into it", t, j)
+                log.append(("Phalf", t, j))
+                b(f"p_half{t}").arrive()
+                yield None  # the second half of the exponentials
+                log.append(("P", t, j))
                 b(f"p_full{t}").arrive()
             if r["active"]:
                 yield ("wait", f"o_full{t}", o_cnt & 1, o_cnt)
@@ -193,12 +208,17 @@ def run(items, stages, rope, seed):
     agents = [producer(), mma(), softmax(0), softmax(1)]
     pending = [None] * 4
     done = [False] * 4
+    stalled = 0
     while not all(done):
         progressed = False
         order = list(range(4))
         rng.shuffle(order)
+        # odd seeds: a random subset of the roles moves in each round, so one
+        # role can run many steps ahead of another (races show up); even
+        # seeds: every role in turn, and a round where none moves is a deadlock
+        subset = seed % 2 == 1
         for a in order:
-            if done[a]:
+            if done[a] or (subset and rng.random() < 0.5):
                 continue
             if pending[a] is not None:
                 _, name, parity, phase = pending[a]
@@ -213,7 +233,8 @@ def run(items, stages, rope, seed):
             except StopIteration:
                 done[a] = True
             progressed = True
-        if not progressed:
+        stalled = 0 if progressed else stalled + 1
+        if (not progressed and not subset) or stalled > 1000:
             raise AssertionError(f"deadlock, waiting on {pending}")
 
 
@@ -240,3 +261,4 @@ ITEM_SETS = {
 def test_two_tile_protocol_finishes_in_order(name, stages, rope):
     for seed in range(25):
         run(ITEM_SETS[name], stages, rope, seed)
+
