@@ -55,11 +55,12 @@ constexpr int kTileN = 128;     // keys per block
 constexpr int kQBlock = 256;    // query rows per work item (two tiles)
 constexpr int kThreads = 384;   // three warpgroups
 // Per-thread registers after setmaxnreg: softmax warpgroups / producer-MMA
-// warpgroup.  The rope kernels' producer and MMA warps keep more state.
-template <bool kRope>
-constexpr uint32_t kSoftmaxRegs = kRope ? 216 : 224;
-template <bool kRope>
-constexpr uint32_t kOtherRegs = kRope ? 72 : 56;
+// warpgroup.  The producer and MMA warps of the rope and ALiBi-ramp kernels
+// keep more state.
+template <bool kMoreOther>
+constexpr uint32_t kSoftmaxRegs = kMoreOther ? 216 : 224;
+template <bool kMoreOther>
+constexpr uint32_t kOtherRegs = kMoreOther ? 72 : 56;
 // setmaxnreg hands out what the launch reserved: 384 threads x 168 registers
 // (the allocation unit is 8 registers per thread; 176 x 384 exceeds 64K)
 static_assert(2 * 128 * kSoftmaxRegs<false> + 128 * kOtherRegs<false> <= (65536 / kThreads) / 8 * 8 * kThreads &&
@@ -104,20 +105,39 @@ enum : int {
 // kRope: queryRope/keyRope with a head dim of 64 — one 128-byte chunk more
 // in every Q tile (after its D columns) and, for K, in a two-slot ring of
 // its own that fills with K under K's barrier.
-template <int D, bool kRope = false>
+// kAug (ALiBi slopes, head dim 64): the column ramp of the ALiBi bias comes
+// out of the S MMA as one more K-step of 16: a chunk after Q's D columns
+// holds, in every row, the slope (over scale) split into three terms, and a
+// fixed chunk holds, for key c of the block, (c, c, c); so S gains
+// slope/scale * c and a block left of every row's diagonal needs no bias
+// work in the softmax (its per-row part joins the max and the shift).
+template <int D, bool kRope = false, bool kAug = false>
 struct Cfg {
     static constexpr int kChunks = D / 64;             // 128-byte swizzle chunks per row
     static constexpr int kChunkBytes = kTileM * 128;   // one chunk of a 128-row tile
     static constexpr int kTileBytes = kTileM * D * 2;  // one K or V tile
-    static constexpr int kQTileBytes = kTileBytes + (kRope ? kChunkBytes : 0);
+    static constexpr int kQTileBytes = kTileBytes + ((kRope || kAug) ? kChunkBytes : 0);
     static constexpr int kRopeSlots = kRope ? 2 : 0;
+    static constexpr int kAugBytes = kAug ? kChunkBytes : 0;  // the fixed (c, c, c) key chunk
     static constexpr int kStages = (D == 128) ? (kRope ? 3 : 4) : 8;  // K/V ring slots
-    static constexpr int kSmemBytes = 2 * kQTileBytes + kStages * kTileBytes + kRopeSlots * kChunkBytes + 1024;
+    static constexpr int kSmemBytes =
+        2 * kQTileBytes + kStages * kTileBytes + kRopeSlots * kChunkBytes + kAugBytes + 1024;
     static constexpr uint32_t kTmemCols = 512;
 };
 constexpr uint32_t kOCol = 256;  // TMEM column of O (S and P use 0..255)
 static_assert(Cfg<128, true>::kSmemBytes + 1024 <= 227 * 1024, "rope tiles exceed shared memory");
 static_assert(Cfg<64, true>::kSmemBytes + 1024 <= 227 * 1024, "rope tiles exceed shared memory");
+static_assert(Cfg<64, false, true>::kSmemBytes + 1024 <= 227 * 1024, "ALiBi ramp chunks exceed shared memory");
+template <int D, int kBias, bool kRope>
+constexpr bool kAugRamp = kBias == 2 && D == 64 && !kRope;
+
+__device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ uint16_t bits16(__half x) { return __half_as_ushort(x); }
+__device__ __forceinline__ uint16_t bits16(__nv_bfloat16 x) { return __bfloat16_as_ushort(x); }
+
+// Row r's 16-byte piece k (k < 8) of a 128-byte-swizzled 128-row chunk.
+__device__ __forceinline__ uint32_t sw128_offset(int r, int k) { return r * 128 + ((k ^ (r & 7)) << 4); }
 
 struct Barriers {
     uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2];
@@ -301,11 +321,11 @@ __device__ __forceinline__ int take_ticket_local(const FaParams& p, Barriers& ba
 // TMA producer (one warp: every lane follows the schedule and waits, so all
 // operands stay warp-uniform; one elected lane issues the copies)
 // ---------------------------------------------------------------------------
-template <int D, bool kRope>
+template <typename T, int D, bool kRope, bool kAug>
 __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
                              const CUtensorMap* tv, const CUtensorMap* tqr, const CUtensorMap* tkr, uint8_t* sQ,
                              uint8_t* sKV, uint8_t* sKr, Barriers& bars, TicketSlots& slots, volatile int* abort) {
-    using C = Cfg<D, kRope>;
+    using C = Cfg<D, kRope, kAug>;
     uint32_t kv_fill = 0, q_fill[2] = {0, 0}, k_sched = 0, kr_fill = 0;
     bool ok = true;
     const int v_chunks = (p.Dv + 63) / 64;
@@ -336,8 +356,25 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
 
         auto load_q = [&](int t) -> bool {
             if (!warp_wait(&bars.q_empty[t], (q_fill[t] & 1) ^ 1, abort, kSiteQEmpty)) return false;
+            if constexpr (kAug) {
+                // the item's slope in every row of the ramp chunk (three terms
+                // whose sum is slope·log2(e)/|scale|, negated with the scale,
+                // as the MMA then negates K), made visible to the tensor core
+                const float a = (p.neg_scale ? -1.f : 1.f) *
+                                static_cast<const float*>(p.pse)[it.b * p.pse_b + it.n * p.pse_n] * kLog2e /
+                                p.scale_log2;
+                const T a0 = static_cast<T>(a);
+                const T a1 = static_cast<T>(a - to_f(a0));
+                const T a2 = static_cast<T>(a - to_f(a0) - to_f(a1));
+                const uint32_t w0 = static_cast<uint32_t>(bits16(a0)) | (static_cast<uint32_t>(bits16(a1)) << 16);
+                const uint32_t w1 = static_cast<uint32_t>(bits16(a2));
+                const uint32_t base = smem_u32(sQ + t * C::kQTileBytes + C::kTileBytes);
+                for (int r = threadIdx.x & 31; r < kTileM; r += 32) st_shared_v4(base + sw128_offset(r, 0), w0, w1, 0u, 0u);
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
             if (elect_one()) {
-                mbar_arrive_expect_tx(&bars.q_full[t], C::kQTileBytes);
+                mbar_arrive_expect_tx(&bars.q_full[t], kAug ? C::kTileBytes : C::kQTileBytes);
                 load_tile(tq, sQ + t * C::kQTileBytes, &bars.q_full[t], it.qb * kQBlock + t * kTileM, it.n, it.b,
                           it.q_off);
                 if constexpr (kRope)
@@ -401,10 +438,10 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
 // warp-uniform values; one elected lane issues each tcgen05 instruction, the
 // same lane every time, so its commits cover its MMAs)
 // ---------------------------------------------------------------------------
-template <typename T, int D, bool kRope>
-__device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* sKr, Barriers& bars,
+template <typename T, int D, bool kRope, bool kAug>
+__device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* sKr, uint8_t* sAug, Barriers& bars,
                         const TicketSlots& slots, uint32_t tmem, volatile int* abort) {
-    using C = Cfg<D, kRope>;
+    using C = Cfg<D, kRope, kAug>;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     const uint32_t idesc_qk = idesc_f16(kBf16, kTileM, kTileN, false, false, p.neg_scale != 0);
     // P·V over the 64-column chunks that hold V's Dv columns
@@ -451,6 +488,10 @@ __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* s
                 const uint64_t qrd = sdesc_sw128(smem_u32(sQ + t * C::kQTileBytes + C::kTileBytes), 1024, 16);
                 const uint64_t krd = sdesc_sw128(smem_u32(sKr + rs * C::kChunkBytes), 1024, 16);
                 mma_ss_k64(tmem + t * kTileN, qrd, krd, idesc_qk, 1u);
+            }
+            if constexpr (kAug) {
+                const uint64_t qad = sdesc_sw128(smem_u32(sQ + t * C::kQTileBytes + C::kTileBytes), 1024, 16);
+                mma_ss(tmem + t * kTileN, qad, sdesc_sw128(smem_u32(sAug), 1024, 16), idesc_qk, 1u);
             }
         }
         __syncwarp();
@@ -715,8 +756,6 @@ __device__ void run_mma_wide(const FaParams& p, uint8_t* sQ, uint8_t* sKV, Barri
 // ---------------------------------------------------------------------------
 // Softmax warpgroup t (128 threads; thread r owns query row r of the tile)
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
-__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 // Two floats rounded to T and packed, `lo` (the lower column) in the low half.
 template <typename T>
@@ -881,6 +920,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tO = tmem + lane_off + kOCol + t * D;
     const float sl2 = p.scale_log2;
+    constexpr bool kAug = !kWide && kBias == 2 && D == 64;  // the ALiBi ramp comes out of the S MMA
     uint32_t s_cnt0 = 0, s_cnt1 = 0, o_cnt = 0, k_sched = 0, g_blk = 0;
     bool ok = true;
 
@@ -944,10 +984,13 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
             float m_blk;
             float row_off = 0.f;  // a per-row bias term kept out of s (added to the max and the shift)
             bool linear = false;
+            bool scaled = kBias == 0;  // s still holds S (the max and the exponentials multiply by sl2)
             if constexpr (kBias == 2) {
                 // A block wholly on one side of every row's diagonal has
                 // -slope·|i - j| = st·c - st·(i - j0) with st = ±slope: a ramp
-                // over the columns plus a per-row constant.
+                // over the columns plus a per-row constant.  With the ramp
+                // from the MMA (kAug: S already holds slope·c / scale) a block
+                // left of the diagonal needs nothing more.
                 const int j0g = j0 + p.alibi_delta;  // key positions relative to the query positions
                 const bool below = j0g + kTileN - 1 <= r0;
                 const bool above = j0g >= r0 + kTileM - 1;
@@ -955,10 +998,14 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                 if (linear) {
                     const float st = below ? slope_l2 : -slope_l2;
                     row_off = -st * (float)(i - j0g);
+                    if (kAug && below) scaled = true;
+                }
+                if (linear && !scaled) {
+                    const float sr = (below ? slope_l2 : -slope_l2) - (kAug ? slope_l2 : 0.f);  // ramp still to apply
                     float t[8];  // ramp at columns c8 + h, four chains of column pairs
 #pragma unroll
-                    for (int h = 0; h < 8; ++h) t[h] = st * (float)h;
-                    const float step = 8.f * st;
+                    for (int h = 0; h < 8; ++h) t[h] = sr * (float)h;
+                    const float step = 8.f * sr;
 #pragma unroll
                     for (int c8 = 0; c8 < kTileN; c8 += 8) {
 #pragma unroll
@@ -976,7 +1023,10 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                     float bias[16];
                     if constexpr (kBias == 2) {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) bias[e] = -slope_l2 * fabsf(fi - (float)(c16 + e));
+                        for (int e = 0; e < 16; ++e) {
+                            const float cf = (float)(c16 + e);
+                            bias[e] = -slope_l2 * (fabsf(fi - cf) + (kAug ? cf : 0.f));
+                        }
                     } else if (pse_row) {
                         load_bias16(pse_row, j0 + c16, pse_cols, pse_vec32, pse_vec, bias);
                     } else {
@@ -1018,7 +1068,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
 #pragma unroll
                     for (int h = 0; h < 8; ++h) mc[h] = max3(mc[h], s[c + 2 * h], s[c + 2 * h + 1]);
                 m_blk = max3(max3(mc[0], mc[1], mc[2]), max3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
-                if constexpr (!kBias) m_blk *= sl2;
+                if (scaled) m_blk *= sl2;
                 m_blk += row_off;
             }
 
@@ -1036,7 +1086,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
             // kPolyPairs of every 8 column pairs take the FMA-pipe exponential
             // (spread over the 8), the others MUFU's ex2
             float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-            const float mult = kBias ? 1.f : sl2;
+            const float mult = scaled ? sl2 : 1.f;
             const float nshift = row_off - shift;
             // Rescale O_t by alpha before this block's P·V reaches it.  Two
             // tiles: O_t is stable, the commit behind this block's S_t covered
@@ -1232,12 +1282,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_qr,
                         const __grid_constant__ CUtensorMap tmap_kr, const FaParams p) {
-    using C = Cfg<D, kRope>;
+    constexpr bool kAug = kAugRamp<D, kBias, kRope>;
+    using C = Cfg<D, kRope, kAug>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
     uint8_t* sKV = smem + 2 * C::kQTileBytes;
     uint8_t* sKr = sKV + C::kStages * C::kTileBytes;
+    uint8_t* sAug = sKr + C::kRopeSlots * C::kChunkBytes;
     __shared__ Barriers bars;
     __shared__ TicketSlots slots;
     __shared__ uint32_t tmem_base;
@@ -1280,21 +1332,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(&tmem_base, C::kTmemCols);
         tmem_relinquish();
     }
+    if constexpr (kAug) {
+        // ALiBi ramp chunks: the Q tiles' ramp chunks zero (the producer
+        // writes each item's slope terms into piece 0 of every row); the
+        // fixed key chunk (c, c, c) in piece 0 of row c, zero elsewhere
+        if (threadIdx.x < 2 * kTileM) {
+            const int t = threadIdx.x / kTileM, r = threadIdx.x % kTileM;
+            const uint32_t qa = smem_u32(sQ + t * C::kQTileBytes + C::kTileBytes) + r * 128;
+            for (int k = 0; k < 8; ++k) st_shared_v4(qa + k * 16, 0u, 0u, 0u, 0u);
+            if (t == 0) {
+                const uint32_t ka = smem_u32(sAug);
+                const uint32_t cc = static_cast<uint32_t>(bits16(static_cast<T>(static_cast<float>(r))));
+                for (int k = 0; k < 8; ++k) st_shared_v4(ka + sw128_offset(r, k), 0u, 0u, 0u, 0u);
+                st_shared_v4(ka + sw128_offset(r, 0), cc | (cc << 16), cc, 0u, 0u);
+            }
+        }
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
 
     if (warp < 8) {
-        setmaxnreg_inc<kSoftmaxRegs<kRope>>();
+        setmaxnreg_inc<kSoftmaxRegs<kRope || kAug>>();
         run_softmax<T, D, kBias>(p, bars, slots, tmem, &abort_flag, warp >> 2);
     } else {
-        setmaxnreg_dec<kOtherRegs<kRope>>();
+        setmaxnreg_dec<kOtherRegs<kRope || kAug>>();
         if (warp == kLoadWarp)
-            run_producer<D, kRope>(p, &tmap_q, &tmap_k, &tmap_v, &tmap_qr, &tmap_kr, sQ, sKV, sKr, bars, slots,
-                                   &abort_flag);
+            run_producer<T, D, kRope, kAug>(p, &tmap_q, &tmap_k, &tmap_v, &tmap_qr, &tmap_kr, sQ, sKV, sKr, bars,
+                                            slots, &abort_flag);
         else if (warp == kMmaWarp)
-            run_mma<T, D, kRope>(p, sQ, sKV, sKr, bars, slots, tmem, &abort_flag);
+            run_mma<T, D, kRope, kAug>(p, sQ, sKV, sKr, sAug, bars, slots, tmem, &abort_flag);
     }
 
     tc_fence_before();
@@ -1389,7 +1458,7 @@ cudaError_t launch_wide(const FaParams& p, const TmaSet& maps, cudaStream_t stre
 
 template <typename T, int D, int kBias, bool kRope = false>
 cudaError_t launch_t(const FaParams& p, const TmaSet& maps, int num_sms, cudaStream_t stream) {
-    using C = Cfg<D, kRope>;
+    using C = Cfg<D, kRope, kAugRamp<D, kBias, kRope>>;
     auto kern = fa_fwd_sm100_kernel<T, D, kBias, kRope>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -1399,7 +1468,8 @@ cudaError_t launch_t(const FaParams& p, const TmaSet& maps, int num_sms, cudaStr
     cudaFuncAttributes attr{};
     e = cudaFuncGetAttributes(&attr, kern);
     if (e != cudaSuccess) return e;
-    if (static_cast<uint64_t>(attr.numRegs) * kThreads < 2ull * 128 * kSoftmaxRegs<kRope> + 128ull * kOtherRegs<kRope>)
+    constexpr bool kMore = kRope || kAugRamp<D, kBias, kRope>;
+    if (static_cast<uint64_t>(attr.numRegs) * kThreads < 2ull * 128 * kSoftmaxRegs<kMore> + 128ull * kOtherRegs<kMore>)
         return cudaErrorLaunchOutOfResources;
     (void)num_sms;
     if (p.grid <= 0) return cudaSuccess;
