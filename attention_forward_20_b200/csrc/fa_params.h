@@ -64,6 +64,7 @@ struct FaParams {
     int32_t st_vec32;           // the 8 lanes of a statistics row allow 32-byte stores
     int32_t mask_vec;           // mask rows allow 16-byte loads
     int32_t pse_vec;            // dense bias rows allow 16-byte loads
+    int32_t pse_tma;            // head dim 64: bias blocks come by TMA (set at launch from TmaSet::pse_ok)
     // dense bias layouts besides [B|1, N|1, Sq, Skv]:
     int32_t pse_rows1024;       // [B|1, N|1, 1024, Skv]: the last 1024 rows of the (lower-triangular) bias
     int32_t pse_flat;           // TND [sum_b N*Sq_b*Skv_b]: each sequence's [N, Sq_b, Skv_b] block in turn
@@ -142,8 +143,12 @@ struct alignas(64) TmaDesc {
 };
 // Q, K, V and (with rope) queryRope, keyRope; without rope qr/kr repeat q/k
 // and are never read.
+// pse: a dense bias tensor [B|1, N|1, Sq, Skv] in boxes of 64 columns x 128
+// rows (pse_ok = 0 when there is none or it is not TMA-legal: the kernel then
+// reads bias rows itself).
 struct TmaSet {
-    TmaDesc q, k, v, qr, kr;
+    TmaDesc q, k, v, qr, kr, pse;
+    int32_t pse_ok;
 };
 
 // Varlen work table of the tcgen05 kernels: one entry {b, qb, q_len, kv_len}

@@ -55,8 +55,8 @@ constexpr int kTileN = 128;     // keys per block
 constexpr int kQBlock = 256;    // query rows per work item (two tiles)
 constexpr int kThreads = 384;   // three warpgroups
 // Per-thread registers after setmaxnreg: softmax warpgroups / producer-MMA
-// warpgroup.  The producer and MMA warps of the rope and ALiBi-ramp kernels
-// keep more state.
+// warpgroup.  The producer and MMA warps of the rope, ALiBi-ramp and
+// bias-buffer kernels keep more state.
 template <bool kMoreOther>
 constexpr uint32_t kSoftmaxRegs = kMoreOther ? 216 : 224;
 template <bool kMoreOther>
@@ -111,7 +111,10 @@ enum : int {
 // fixed chunk holds, for key c of the block, (c, c, c); so S gains
 // slope/scale * c and a block left of every row's diagonal needs no bias
 // work in the softmax (its per-row part joins the max and the shift).
-template <int D, bool kRope = false, bool kAug = false>
+// kTmaBias (dense bias tensor, head dim 64): the bias block of each query
+// tile comes into shared memory by TMA (two 64-column boxes, two buffers per
+// tile) instead of per-thread row loads; the K/V ring has 4 slots then.
+template <int D, bool kRope = false, bool kAug = false, bool kTmaBias = false>
 struct Cfg {
     static constexpr int kChunks = D / 64;             // 128-byte swizzle chunks per row
     static constexpr int kChunkBytes = kTileM * 128;   // one chunk of a 128-row tile
@@ -119,17 +122,22 @@ struct Cfg {
     static constexpr int kQTileBytes = kTileBytes + ((kRope || kAug) ? kChunkBytes : 0);
     static constexpr int kRopeSlots = kRope ? 2 : 0;
     static constexpr int kAugBytes = kAug ? kChunkBytes : 0;  // the fixed (c, c, c) key chunk
-    static constexpr int kStages = (D == 128) ? (kRope ? 3 : 4) : 8;  // K/V ring slots
+    static constexpr int kStages = (D == 128) ? (kRope ? 3 : 4) : (kTmaBias ? 4 : 8);  // K/V ring slots
+    static constexpr int kBiasTileBytes = kTileM * kTileN * 2;                     // one 128 x 128 block
+    static constexpr int kBiasBytes = kTmaBias ? 4 * kBiasTileBytes : 0;          // 2 tiles x 2 buffers
     static constexpr int kSmemBytes =
-        2 * kQTileBytes + kStages * kTileBytes + kRopeSlots * kChunkBytes + kAugBytes + 1024;
+        2 * kQTileBytes + kStages * kTileBytes + kRopeSlots * kChunkBytes + kAugBytes + kBiasBytes + 1024;
     static constexpr uint32_t kTmemCols = 512;
 };
 constexpr uint32_t kOCol = 256;  // TMEM column of O (S and P use 0..255)
 static_assert(Cfg<128, true>::kSmemBytes + 1024 <= 227 * 1024, "rope tiles exceed shared memory");
 static_assert(Cfg<64, true>::kSmemBytes + 1024 <= 227 * 1024, "rope tiles exceed shared memory");
 static_assert(Cfg<64, false, true>::kSmemBytes + 1024 <= 227 * 1024, "ALiBi ramp chunks exceed shared memory");
+static_assert(Cfg<64, false, false, true>::kSmemBytes + 1024 <= 227 * 1024, "bias buffers exceed shared memory");
 template <int D, int kBias, bool kRope>
 constexpr bool kAugRamp = kBias == 2 && D == 64 && !kRope;
+template <int D, int kBias, bool kRope>
+constexpr bool kTmaBiasK = kBias == 1 && D == 64 && !kRope;
 
 __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -142,6 +150,7 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int k) { return r * 128 
 struct Barriers {
     uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2];
     uint64_t p_half[2];    // two-tile kernel: the first 64 keys' half of P_t is in TMEM
+    uint64_t bias_full[2][2], bias_empty[2][2];  // kTmaBias: tile t's bias buffers
     uint64_t kv_full[8], kv_empty[8];
     uint64_t kr_empty[2];  // keyRope slots (the K load's kv_full also covers its keyRope chunk)
     uint64_t pv_done;      // wide kernel: one completion per key block's P·V
@@ -321,12 +330,13 @@ __device__ __forceinline__ int take_ticket_local(const FaParams& p, Barriers& ba
 // TMA producer (one warp: every lane follows the schedule and waits, so all
 // operands stay warp-uniform; one elected lane issues the copies)
 // ---------------------------------------------------------------------------
-template <typename T, int D, bool kRope, bool kAug>
+template <typename T, int D, bool kRope, bool kAug, bool kTmaBias>
 __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
-                             const CUtensorMap* tv, const CUtensorMap* tqr, const CUtensorMap* tkr, uint8_t* sQ,
-                             uint8_t* sKV, uint8_t* sKr, Barriers& bars, TicketSlots& slots, volatile int* abort) {
-    using C = Cfg<D, kRope, kAug>;
-    uint32_t kv_fill = 0, q_fill[2] = {0, 0}, k_sched = 0, kr_fill = 0;
+                             const CUtensorMap* tv, const CUtensorMap* tqr, const CUtensorMap* tkr,
+                             const CUtensorMap* tpse, uint8_t* sQ, uint8_t* sKV, uint8_t* sKr, uint8_t* sBias,
+                             Barriers& bars, TicketSlots& slots, volatile int* abort) {
+    using C = Cfg<D, kRope, kAug, kTmaBias>;
+    uint32_t kv_fill = 0, q_fill[2] = {0, 0}, k_sched = 0, kr_fill = 0, b_fill[2] = {0, 0};
     bool ok = true;
     const int v_chunks = (p.Dv + 63) / 64;
 
@@ -412,10 +422,38 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
             return true;
         };
 
+        // kTmaBias: tile t's bias block [rows of the tile] x [128 keys of
+        // block jb] into its next buffer (broadcast dimensions read index 0)
+        auto load_bias = [&](int t, int jb) -> bool {
+            const uint32_t slot = b_fill[t] & 1;
+            if (!warp_wait(&bars.bias_empty[t][slot], ((b_fill[t] >> 1) & 1) ^ 1, abort, kSiteKvEmpty)) return false;
+            if (elect_one()) {
+                uint8_t* dst = sBias + (t * 2 + slot) * C::kBiasTileBytes;
+                const int row = it.qb * kQBlock + t * kTileM;
+                const int nb = p.pse_n ? it.n : 0, bb = p.pse_b ? it.b : 0;
+                // the second box only when it starts inside the keys (columns
+                // past the keys are masked; the first box always starts inside)
+                const bool second = jb * kTileN + 64 < p.Skv;
+                mbar_arrive_expect_tx(&bars.bias_full[t][slot], second ? C::kBiasTileBytes : C::kBiasTileBytes / 2);
+                tma_load_4d(dst, tpse, &bars.bias_full[t][slot], jb * kTileN, row, nb, bb);
+                if (second)
+                    tma_load_4d(dst + C::kBiasTileBytes / 2, tpse, &bars.bias_full[t][slot], jb * kTileN + 64, row, nb,
+                                bb);
+            }
+            __syncwarp();
+            ++b_fill[t];
+            return true;
+        };
+
         if (tr[0].active() && !load_q(0)) { ok = false; break; }
         for (int jb = lo; ok && jb <= hi; ++jb) {
             if (!load_kv(tk, jb, true)) { ok = false; break; }
             if (jb == lo && tr[1].active() && !load_q(1)) { ok = false; break; }
+            if (kTmaBias && p.pse_tma) {
+                for (int t = 0; t < 2 && ok; ++t)
+                    if (tr[t].has(jb) && !load_bias(t, jb)) ok = false;
+                if (!ok) break;
+            }
             if (!load_kv(tv, jb, false)) { ok = false; break; }
         }
     }
@@ -431,6 +469,12 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
     }
     for (int t = 0; t < 2; ++t)
         if (q_fill[t]) mbar_wait_drain(&bars.q_full[t], (q_fill[t] - 1) & 1, abort, kSiteDrain);
+    for (int t = 0; t < 2; ++t)
+        for (uint32_t k = 0; k < 2; ++k)
+            if (k < b_fill[t]) {
+                const uint32_t last = b_fill[t] - 1 - ((b_fill[t] - 1 - k) % 2);
+                mbar_wait_drain(&bars.bias_full[t][k], (last >> 1) & 1, abort, kSiteDrain);
+            }
 }
 
 // ---------------------------------------------------------------------------
@@ -438,10 +482,10 @@ __device__ void run_producer(const FaParams& p, const CUtensorMap* tq, const CUt
 // warp-uniform values; one elected lane issues each tcgen05 instruction, the
 // same lane every time, so its commits cover its MMAs)
 // ---------------------------------------------------------------------------
-template <typename T, int D, bool kRope, bool kAug>
+template <typename T, int D, bool kRope, bool kAug, bool kTmaBias>
 __device__ void run_mma(const FaParams& p, uint8_t* sQ, uint8_t* sKV, uint8_t* sKr, uint8_t* sAug, Barriers& bars,
                         const TicketSlots& slots, uint32_t tmem, volatile int* abort) {
-    using C = Cfg<D, kRope, kAug>;
+    using C = Cfg<D, kRope, kAug, kTmaBias>;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     const uint32_t idesc_qk = idesc_f16(kBf16, kTileM, kTileN, false, false, p.neg_scale != 0);
     // P·V over the 64-column chunks that hold V's Dv columns
@@ -914,15 +958,16 @@ __device__ __forceinline__ void store_stats(const FaParams& p, const Item& it, i
 // kOCol, and a rescale of O first waits for the previous block's P·V (pv_done).
 template <typename T, int D, int kBias, bool kWide = false>
 __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots& slots, uint32_t tmem,
-                            volatile int* abort, int t) {
+                            volatile int* abort, int t, uint8_t* sBias = nullptr) {
     const int quad = (threadIdx.x >> 5) & 3;
     const int row = quad * 32 + (threadIdx.x & 31);
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tO = tmem + lane_off + kOCol + t * D;
     const float sl2 = p.scale_log2;
     constexpr bool kAug = !kWide && kBias == 2 && D == 64;  // the ALiBi ramp comes out of the S MMA
-    uint32_t s_cnt0 = 0, s_cnt1 = 0, o_cnt = 0, k_sched = 0, g_blk = 0;
+    uint32_t s_cnt0 = 0, s_cnt1 = 0, o_cnt = 0, k_sched = 0, g_blk = 0, bf_cnt = 0;
     bool ok = true;
+    const bool tma_bias = kBias == 1 && sBias != nullptr && p.pse_tma;  // bias blocks in shared memory
 
     while (ok) {
         Item tit;
@@ -958,7 +1003,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
             if constexpr (kBias == 1) {
                 // the next block's bias row segment (256 bytes) on its way to L2
                 const int jn = (jb + 1) * kTileN;
-                if (pse_row && jb < tr.hi && jn < pse_cols) {
+                if (pse_row && !tma_bias && jb < tr.hi && jn < pse_cols) {
                     prefetch_l2(pse_row + jn);
                     if (jn + 64 < pse_cols) prefetch_l2(pse_row + jn + 64);
                 }
@@ -1016,6 +1061,12 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                     }
                 }
             }
+            uint32_t brow = 0;  // this thread's row of the block's bias buffer (tma_bias)
+            if (tma_bias) {
+                const uint32_t slot = bf_cnt & 1;
+                if (!warp_wait(&bars.bias_full[t][slot], (bf_cnt >> 1) & 1, abort, kSiteKvFull)) { ok = false; break; }
+                brow = smem_u32(sBias + (t * 2 + slot) * (kTileM * kTileN * 2)) + row * 128;
+            }
             if (kBias && !linear) {
                 const float fi = (float)(i - j0 - p.alibi_delta);
 #pragma unroll
@@ -1027,6 +1078,16 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                             const float cf = (float)(c16 + e);
                             bias[e] = -slope_l2 * (fabsf(fi - cf) + (kAug ? cf : 0.f));
                         }
+                    } else if (tma_bias) {
+                        // two 16-byte pieces of the row in a 128-byte-swizzled 64-column box
+#pragma unroll
+                        for (int k2 = 0; k2 < 2; ++k2) {
+                            const int k = ((c16 & 63) >> 3) + k2;
+                            const uint4 u = ld_shared_v4(brow + (c16 >> 6) * (kTileM * 128) + ((k ^ (row & 7)) << 4));
+                            const T* h = reinterpret_cast<const T*>(&u);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) bias[8 * k2 + e] = to_f(h[e]) * kLog2e;
+                        }
                     } else if (pse_row) {
                         load_bias16(pse_row, j0 + c16, pse_cols, pse_vec32, pse_vec, bias);
                     } else {
@@ -1036,6 +1097,10 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
 #pragma unroll
                     for (int e = 0; e < 16; ++e) s[c16 + e] = fmaf(s[c16 + e], sl2, bias[e]);
                 }
+            }
+            if (tma_bias) {  // the buffer may be refilled
+                mbar_arrive(&bars.bias_empty[t][bf_cnt & 1]);
+                ++bf_cnt;
             }
             if (!full) {
                 // keys of this row kept by the sequence end and the band:
@@ -1281,15 +1346,18 @@ template <typename T, int D, int kBias, bool kRope>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_qr,
-                        const __grid_constant__ CUtensorMap tmap_kr, const FaParams p) {
+                        const __grid_constant__ CUtensorMap tmap_kr, const __grid_constant__ CUtensorMap tmap_pse,
+                        const FaParams p) {
     constexpr bool kAug = kAugRamp<D, kBias, kRope>;
-    using C = Cfg<D, kRope, kAug>;
+    constexpr bool kTmaBias = kTmaBiasK<D, kBias, kRope>;
+    using C = Cfg<D, kRope, kAug, kTmaBias>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
     uint8_t* sKV = smem + 2 * C::kQTileBytes;
     uint8_t* sKr = sKV + C::kStages * C::kTileBytes;
     uint8_t* sAug = sKr + C::kRopeSlots * C::kChunkBytes;
+    uint8_t* sBias = sAug + C::kAugBytes;
     __shared__ Barriers bars;
     __shared__ TicketSlots slots;
     __shared__ uint32_t tmem_base;
@@ -1303,6 +1371,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars.s_full[t], 1);
             mbar_init(&bars.p_full[t], kTileM);
             mbar_init(&bars.p_half[t], kTileM);
+            for (int k = 0; k < 2; ++k) {
+                mbar_init(&bars.bias_full[t][k], 1);
+                mbar_init(&bars.bias_empty[t][k], kTileM);
+            }
             mbar_init(&bars.o_full[t], 1);
         }
         for (int s = 0; s < C::kStages; ++s) {
@@ -1327,6 +1399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&tmap_qr);
             prefetch_tmap(&tmap_kr);
         }
+        if (kTmaBias && p.pse_tma) prefetch_tmap(&tmap_pse);
     }
     if (warp == kMmaWarp) {
         tmem_alloc(&tmem_base, C::kTmemCols);
@@ -1355,15 +1428,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = tmem_base;
 
     if (warp < 8) {
-        setmaxnreg_inc<kSoftmaxRegs<kRope || kAug>>();
-        run_softmax<T, D, kBias>(p, bars, slots, tmem, &abort_flag, warp >> 2);
+        setmaxnreg_inc<kSoftmaxRegs<kRope || kAug || kTmaBias>>();
+        run_softmax<T, D, kBias>(p, bars, slots, tmem, &abort_flag, warp >> 2, kTmaBias ? sBias : nullptr);
     } else {
-        setmaxnreg_dec<kOtherRegs<kRope || kAug>>();
+        setmaxnreg_dec<kOtherRegs<kRope || kAug || kTmaBias>>();
         if (warp == kLoadWarp)
-            run_producer<T, D, kRope, kAug>(p, &tmap_q, &tmap_k, &tmap_v, &tmap_qr, &tmap_kr, sQ, sKV, sKr, bars,
-                                            slots, &abort_flag);
+            run_producer<T, D, kRope, kAug, kTmaBias>(p, &tmap_q, &tmap_k, &tmap_v, &tmap_qr, &tmap_kr, &tmap_pse, sQ,
+                                                      sKV, sKr, sBias, bars, slots, &abort_flag);
         else if (warp == kMmaWarp)
-            run_mma<T, D, kRope, kAug>(p, sQ, sKV, sKr, sAug, bars, slots, tmem, &abort_flag);
+            run_mma<T, D, kRope, kAug, kTmaBias>(p, sQ, sKV, sKr, sAug, bars, slots, tmem, &abort_flag);
     }
 
     tc_fence_before();
@@ -1458,7 +1531,7 @@ cudaError_t launch_wide(const FaParams& p, const TmaSet& maps, cudaStream_t stre
 
 template <typename T, int D, int kBias, bool kRope = false>
 cudaError_t launch_t(const FaParams& p, const TmaSet& maps, int num_sms, cudaStream_t stream) {
-    using C = Cfg<D, kRope, kAugRamp<D, kBias, kRope>>;
+    using C = Cfg<D, kRope, kAugRamp<D, kBias, kRope>, kTmaBiasK<D, kBias, kRope>>;
     auto kern = fa_fwd_sm100_kernel<T, D, kBias, kRope>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -1468,14 +1541,16 @@ cudaError_t launch_t(const FaParams& p, const TmaSet& maps, int num_sms, cudaStr
     cudaFuncAttributes attr{};
     e = cudaFuncGetAttributes(&attr, kern);
     if (e != cudaSuccess) return e;
-    constexpr bool kMore = kRope || kAugRamp<D, kBias, kRope>;
+    constexpr bool kMore = kRope || kAugRamp<D, kBias, kRope> || kTmaBiasK<D, kBias, kRope>;
     if (static_cast<uint64_t>(attr.numRegs) * kThreads < 2ull * 128 * kSoftmaxRegs<kMore> + 128ull * kOtherRegs<kMore>)
         return cudaErrorLaunchOutOfResources;
     (void)num_sms;
     if (p.grid <= 0) return cudaSuccess;
     auto map = [](const TmaDesc& d) -> const CUtensorMap& { return *reinterpret_cast<const CUtensorMap*>(&d); };
+    FaParams pl = p;
+    pl.pse_tma = (kTmaBiasK<D, kBias, kRope> && maps.pse_ok) ? 1 : 0;
     kern<<<p.grid, kThreads, C::kSmemBytes, stream>>>(map(maps.q), map(maps.k), map(maps.v), map(maps.qr),
-                                                      map(maps.kr), p);
+                                                      map(maps.kr), map(maps.pse), pl);
     e = cudaGetLastError();
     if (e != cudaSuccess || p.n_pieces == 0) return e;
     const int n_split = (p.n_tickets - p.n_whole) / p.n_pieces;
@@ -1576,6 +1651,28 @@ cudaError_t make_sm100_tmaps(const FaParams& p, TmaSet* maps) {
     if (e == cudaSuccess) e = encode(&maps->k, p, p.k, p.D, p.Tkv, p.Nkv, p.k_s, p.k_n, p.k_b);
     if (e == cudaSuccess) e = encode(&maps->v, p, p.v, p.Dv, p.Tkv, p.Nkv, p.v_s, p.v_n, p.v_b);
     if (e != cudaSuccess) return e;
+    // a dense bias [B|1, N|1, Sq, Skv] (not the compressed or flattened forms):
+    // 64 x 128 boxes for the head-dim-64 kernels' bias buffers
+    maps->pse = maps->q;
+    maps->pse_ok = 0;
+    if (p.pse_type == 1 && !p.pse_rows1024 && !p.pse_flat && !p.varlen &&
+        (reinterpret_cast<uintptr_t>(p.pse) & 15u) == 0 && p.pse_i % 8 == 0 && p.pse_n % 8 == 0 && p.pse_b % 8 == 0) {
+        EncodeTiledFn fn = encode_fn();
+        const cuuint64_t nb = p.pse_n ? (cuuint64_t)p.Nq : 1, bb = p.pse_b ? (cuuint64_t)p.B : 1;
+        const cuuint64_t dims[4] = {(cuuint64_t)p.Skv, (cuuint64_t)p.Sq, nb, bb};
+        const cuuint64_t strides[3] = {stride_bytes(p.pse_i, p.Sq), p.pse_n ? (cuuint64_t)p.pse_n * 2 : 16,
+                                       p.pse_b ? (cuuint64_t)p.pse_b * 2 : 16};
+        const cuuint32_t box[4] = {64, 128, 1, 1};
+        const cuuint32_t es[4] = {1, 1, 1, 1};
+        const CUtensorMapDataType dt =
+            p.dtype == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+        if (fn && fn(reinterpret_cast<CUtensorMap*>(&maps->pse), dt, 4, const_cast<void*>(p.pse), dims, strides, box,
+                     es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            maps->pse_ok = 1;
+        else
+            maps->pse = maps->q;
+    }
     if (p.Dr) {
         e = encode(&maps->qr, p, p.qr, p.Dr, p.Tq, p.Nq, p.qr_s, p.qr_n, p.qr_b);
         if (e == cudaSuccess) e = encode(&maps->kr, p, p.kr, p.Dr, p.Tkv, p.Nkv, p.kr_s, p.kr_n, p.kr_b);

@@ -139,6 +139,26 @@ def test_dense_pse_tensor(dtype):
     compare_full(w)
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_dense_pse_tensor_staged_by_tma(dtype):
+    """Head dim 64 with a dense bias whose rows are 16-byte multiples: the
+    bias blocks come into shared memory by TMA (two buffers per query tile).
+    Ragged query and key tails, a band, bias broadcast over batch or heads,
+    and fewer queries than keys."""
+    s = 392  # 3 blocks + 8 rows
+    w = W("BNSD", dtype, (2, 2, s, 64), 2, 520, pre_tokens=200, next_tokens=30)
+    w.pse, w.pse_type = normal((2, 2, s, s), dtype, 525), 1
+    compare_full(w)
+    w.pse = normal((1, 2, s, s), dtype, 526)   # broadcast over the batch
+    compare_full(w)
+    w.pse = normal((2, 1, s, s), dtype, 527)   # broadcast over the heads
+    w.next_tokens = 0
+    compare_full(w)
+    w = W("BSND", dtype, (1, 300, 2, 64), 2, 530, kshape=(1, 392, 2, 64), sink=normal((2,), "f32", 534))
+    w.pse, w.pse_type = normal((1, 2, 300, 392), dtype, 535), 1
+    compare_full(w)
+
+
 def test_sq_differs_from_skv():
     w = W("BNSD", "f16", (2, 2, 200, 128), 2, 600, kshape=(2, 2, 333, 128))
     compare_full(w)
