@@ -138,6 +138,10 @@ template <int D, int kBias, bool kRope>
 constexpr bool kAugRamp = kBias == 2 && D == 64 && !kRope;
 template <int D, int kBias, bool kRope>
 constexpr bool kTmaBiasK = kBias == 1 && D == 64 && !kRope;
+// compressed-bias windows (in the bias buffers): 160 fp32 per copy, 4 copies per warp
+constexpr int kWinLen = 160;
+constexpr int kWinBytes = 4 * kWinLen * 4;
+static_assert(8 * kWinBytes <= 4 * kTileM * kTileN * 2, "windows exceed the bias buffers");
 
 __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -1067,6 +1071,42 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                 if (!warp_wait(&bars.bias_full[t][slot], (bf_cnt >> 1) & 1, abort, kSiteKvFull)) { ok = false; break; }
                 brow = smem_u32(sBias + (t * 2 + slot) * (kTileM * kTileN * 2)) + row * 128;
             }
+            // Compressed bias, a warp whose 32 rows all lie above the stored
+            // rows: row i reads stored row 0 at column j + first - i, so the
+            // warp needs 159 consecutive stored values per key block.  They
+            // go to shared memory (in the bias buffers, unused for this bias
+            // form) as fp32 times log2(e), in four copies shifted by 0..3
+            // values, so that every row's 128 values are four-aligned runs
+            // of one copy.
+            uint32_t wrow = 0;  // this thread's run in the warp's window (0: no window)
+            if (kBias == 1 && sBias != nullptr && p.pse_rows1024) {
+                const int first = it.q_len - 1024;
+                const int w0 = r0 + quad * 32;
+                if (w0 + 31 < first) {
+                    const int lane = threadIdx.x & 31;
+                    const uint32_t wbase = smem_u32(sBias + (t * 4 + quad) * kWinBytes);
+                    const T* srow = static_cast<const T*>(p.pse) + it.b * p.pse_b + it.n * p.pse_n;
+                    const int col0 = j0 + first - w0 - 31;  // stored column of window value 0
+                    __syncwarp();  // every lane has read the previous block's window
+#pragma unroll
+                    for (int m = 0; m < 6; ++m) {
+                        const int x = lane + 32 * m;
+                        if (x < kWinLen + 3) {
+                            const int col = col0 + x;
+                            const float g = (col >= 0 && col < it.kv_len) ? to_f(srow[col]) * kLog2e : 0.f;
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                if (x - k >= 0 && x - k < kWinLen)
+                                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(wbase + (k * kWinLen + x - k) * 4),
+                                                 "f"(g)
+                                                 : "memory");
+                        }
+                    }
+                    __syncwarp();
+                    const int x0 = 31 - lane;  // this row's first window value
+                    wrow = wbase + ((x0 & 3) * kWinLen + (x0 & ~3)) * 4;
+                }
+            }
             if (kBias && !linear) {
                 const float fi = (float)(i - j0 - p.alibi_delta);
 #pragma unroll
@@ -1087,6 +1127,15 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                             const T* h = reinterpret_cast<const T*>(&u);
 #pragma unroll
                             for (int e = 0; e < 8; ++e) bias[8 * k2 + e] = to_f(h[e]) * kLog2e;
+                        }
+                    } else if (wrow) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const uint4 u = ld_shared_v4(wrow + (c16 + 4 * q4) * 4);
+                            bias[4 * q4] = __uint_as_float(u.x);
+                            bias[4 * q4 + 1] = __uint_as_float(u.y);
+                            bias[4 * q4 + 2] = __uint_as_float(u.z);
+                            bias[4 * q4 + 3] = __uint_as_float(u.w);
                         }
                     } else if (pse_row) {
                         load_bias16(pse_row, j0 + c16, pse_cols, pse_vec32, pse_vec, bias);

@@ -520,11 +520,14 @@ def test_compressed_alibi_bias(dtype, d):
     compare_full(w)
 
 
-def test_compressed_bias_not_translation_invariant():
-    # arbitrary stored values: the kernel must read them as the oracle's reading says
-    s, n = 1090, 2
-    w = W("BSND", "bf16", (2, s, n, 128), n, 3310, next_tokens=0)
-    w.pse = normal((2, n, 1024, s), "bf16", 3315)
+@pytest.mark.parametrize("dtype,d,s", [("bf16", 128, 1090), ("f16", 64, 1300), ("bf16", 64, 1091)])
+def test_compressed_bias_not_translation_invariant(dtype, d, s):
+    # arbitrary stored values: the kernel must read them as the oracle's reading
+    # says (head dim 64: rows above the stored ones through the per-warp
+    # windows, including a warp that straddles the first stored row)
+    n = 2
+    w = W("BSND", dtype, (2, s, n, d), n, 3310, next_tokens=0, pre_tokens=700)
+    w.pse = normal((2, n, 1024, s), dtype, 3315)
     w.pse_type = 1
     compare_full(w)
 
