@@ -1039,10 +1039,14 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                 // -slope·|i - j| = st·c - st·(i - j0) with st = ±slope: a ramp
                 // over the columns plus a per-row constant.  With the ramp
                 // from the MMA (kAug: S already holds slope·c / scale) a block
-                // left of the diagonal needs nothing more.
+                // left of the diagonal needs nothing more.  When the band
+                // keeps no key right of a row's diagonal (next + delta <= 0,
+                // so j + delta <= i for every kept key), every block is
+                // "below" for the keys it keeps, the diagonal block as well:
+                // the keys past the diagonal are masked out anyway.
                 const int j0g = j0 + p.alibi_delta;  // key positions relative to the query positions
-                const bool below = j0g + kTileN - 1 <= r0;
-                const bool above = j0g >= r0 + kTileM - 1;
+                const bool below = j0g + kTileN - 1 <= r0 || (int64_t)p.next + p.alibi_delta <= 0;
+                const bool above = !below && (j0g >= r0 + kTileM - 1 || (int64_t)p.alibi_delta - p.pre >= 0);
                 linear = below || above;
                 if (linear) {
                     const float st = below ? slope_l2 : -slope_l2;

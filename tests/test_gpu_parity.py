@@ -89,6 +89,18 @@ def test_band_alibi_two_sided():
     compare_full(w)
 
 
+@pytest.mark.parametrize("dtype,d,pre,nxt", [("f16", 64, 0, 200), ("bf16", 128, -3, 150), ("f16", 256, 0, 90),
+                                             ("bf16", 64, 260, -2), ("f16", 128, 300, 0)])
+def test_band_alibi_one_side_of_diagonal(dtype, d, pre, nxt):
+    """Bands that keep keys on one side of the diagonal only (preTokens <= 0:
+    at or right of it; nextTokens <= 0: at or left of it), so that the ALiBi
+    distance |i - j| is linear in j over every kept key of every block, the
+    diagonal block included (V5 page: preTokens/nextTokens, pseType 2)."""
+    w = W("BNSD", dtype, (2, 3, 330, d), 3, 610 + d, pre_tokens=pre, next_tokens=nxt,
+          pse=alibi_slopes(3), pse_type=2)
+    compare_full(w)
+
+
 def _per_batch_slopes(n_batch, n_heads):
     """fp32 [B, N] ALiBi slopes, different along both axes and not symmetric."""
     b = torch.arange(n_batch, dtype=torch.float64)[:, None]
