@@ -1160,6 +1160,12 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                 // columns [c_lo, c_hi] of the block (empty when c_hi < c_lo)
                 const int c_lo = max(0, i - p.pre - j0);
                 const int c_hi = min(min(kTileN - 1, it.kv_len - 1 - j0), i + p.next - j0);
+                // kept: 0 <= c - c_lo <= c_hi - c_lo, one unsigned compare
+                // (nothing kept: c - (kTileN + 1) wraps above a span of 0)
+                const bool any = c_hi >= c_lo;
+                const uint32_t span = any ? static_cast<uint32_t>(c_hi - c_lo) : 0u;
+                const int base = any ? c_lo : kTileN + 1;
+                const bool lo_zero = __all_sync(0xffffffffu, c_lo == 0);  // every lane (mask_row may differ)
                 if (mask_row) {
 #pragma unroll
                     for (int c16 = 0; c16 < kTileN; c16 += 16) {
@@ -1167,13 +1173,19 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             const int c = c16 + e;
-                            if (c < c_lo || c > c_hi || ((excl >> e) & 1u)) s[c] = -CUDART_INF_F;
+                            const bool keep = static_cast<uint32_t>(c - base) <= span && ((excl >> e) & 1u) == 0u;
+                            s[c] = keep ? s[c] : -CUDART_INF_F;
                         }
                     }
+                } else if (lo_zero) {
+                    // the usual partial block (a causal diagonal, the keys'
+                    // end): one compare and one select per column
+#pragma unroll
+                    for (int c = 0; c < kTileN; ++c) s[c] = c <= c_hi ? s[c] : -CUDART_INF_F;
                 } else {
 #pragma unroll
                     for (int c = 0; c < kTileN; ++c)
-                        if (c < c_lo || c > c_hi) s[c] = -CUDART_INF_F;
+                        s[c] = static_cast<uint32_t>(c - base) <= span ? s[c] : -CUDART_INF_F;
                 }
             }
             {
