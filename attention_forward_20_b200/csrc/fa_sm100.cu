@@ -814,21 +814,21 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
         return pack_f16x2(lo, hi);
 }
 
-// Additive bias of 8 consecutive keys starting at j from a dense pse row (query dtype), times log2(e).
+// Additive bias of 8 consecutive keys starting at j from a dense pse row (query dtype), in natural units.
 template <typename T>
 __device__ __forceinline__ void load_bias8(const T* row, int j, int kv_len, bool vec, float* out) {
     if (vec && j + 8 <= kv_len) {
         const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + j));
         const T* h = reinterpret_cast<const T*>(&u);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) out[e] = to_f(h[e]) * kLog2e;
+        for (int e = 0; e < 8; ++e) out[e] = to_f(h[e]);
     } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) out[e] = (j + e < kv_len) ? to_f(row[j + e]) * kLog2e : 0.f;
+        for (int e = 0; e < 8; ++e) out[e] = (j + e < kv_len) ? to_f(row[j + e]) : 0.f;
     }
 }
 
-// Additive bias of 16 consecutive keys starting at j (times log2(e)): one
+// Additive bias of 16 consecutive keys starting at j (natural units): one
 // 32-byte load when the row allows it, else two 8-key loads.
 template <typename T>
 __device__ __forceinline__ void load_bias16(const T* row, int j, int kv_len, bool vec32, bool vec, float* out) {
@@ -837,7 +837,7 @@ __device__ __forceinline__ void load_bias16(const T* row, int j, int kv_len, boo
         ld_global_nc_v8(row + j, w);
         const T* h = reinterpret_cast<const T*>(w);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) out[e] = to_f(h[e]) * kLog2e;
+        for (int e = 0; e < 16; ++e) out[e] = to_f(h[e]);
     } else {
         load_bias8(row, j, kv_len, vec, out);
         load_bias8(row, j + 8, kv_len, vec, out + 8);
@@ -968,6 +968,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tO = tmem + lane_off + kOCol + t * D;
     const float sl2 = p.scale_log2;
+    const float abs_scale = fabsf(p.scale);  // the MMA negates K for a negative scale
     constexpr bool kAug = !kWide && kBias == 2 && D == 64;  // the ALiBi ramp comes out of the S MMA
     uint32_t s_cnt0 = 0, s_cnt1 = 0, o_cnt = 0, k_sched = 0, g_blk = 0, bf_cnt = 0;
     bool ok = true;
@@ -1034,6 +1035,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
             float row_off = 0.f;  // a per-row bias term kept out of s (added to the max and the shift)
             bool linear = false;
             bool scaled = kBias == 0;  // s still holds S (the max and the exponentials multiply by sl2)
+            // after the bias: s in log2 units (ALiBi), natural units (bias tensor)
             if constexpr (kBias == 2) {
                 // A block wholly on one side of every row's diagonal has
                 // -slope·|i - j| = st·c - st·(i - j0) with st = ±slope: a ramp
@@ -1097,7 +1099,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                         const int x = lane + 32 * m;
                         if (x < kWinLen + 3) {
                             const int col = col0 + x;
-                            const float g = (col >= 0 && col < it.kv_len) ? to_f(srow[col]) * kLog2e : 0.f;
+                            const float g = (col >= 0 && col < it.kv_len) ? to_f(srow[col]) : 0.f;
 #pragma unroll
                             for (int k = 0; k < 4; ++k)
                                 if (x - k >= 0 && x - k < kWinLen)
@@ -1130,7 +1132,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                             const uint4 u = ld_shared_v4(brow + (c16 >> 6) * (kTileM * 128) + ((k ^ (row & 7)) << 4));
                             const T* h = reinterpret_cast<const T*>(&u);
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) bias[8 * k2 + e] = to_f(h[e]) * kLog2e;
+                            for (int e = 0; e < 8; ++e) bias[8 * k2 + e] = to_f(h[e]);
                         }
                     } else if (wrow) {
 #pragma unroll
@@ -1147,8 +1149,10 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
 #pragma unroll
                         for (int e = 0; e < 16; ++e) bias[e] = 0.f;
                     }
+                    // ALiBi terms are in log2 units; a bias tensor's are
+                    // natural, so its scores stay natural (unit = log2 e)
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) s[c16 + e] = fmaf(s[c16 + e], sl2, bias[e]);
+                    for (int e = 0; e < 16; ++e) s[c16 + e] = fmaf(s[c16 + e], kBias == 2 ? sl2 : abs_scale, bias[e]);
                 }
             }
             if (tma_bias) {  // the buffer may be refilled
@@ -1199,6 +1203,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                     for (int h = 0; h < 8; ++h) mc[h] = max3(mc[h], s[c + 2 * h], s[c + 2 * h + 1]);
                 m_blk = max3(max3(mc[0], mc[1], mc[2]), max3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
                 if (scaled) m_blk *= sl2;
+                if (kBias == 1) m_blk *= kLog2e;
                 m_blk += row_off;
             }
 
@@ -1216,7 +1221,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
             // kPolyPairs of every 8 column pairs take the FMA-pipe exponential
             // (spread over the 8), the others MUFU's ex2
             float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-            const float mult = scaled ? sl2 : 1.f;
+            const float mult = scaled ? sl2 : (kBias == 1 ? kLog2e : 1.f);
             const float nshift = row_off - shift;
             // Rescale O_t by alpha before this block's P·V reaches it.  Two
             // tiles: O_t is stable, the commit behind this block's S_t covered
