@@ -147,6 +147,12 @@ __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ uint16_t bits16(__half x) { return __half_as_ushort(x); }
 __device__ __forceinline__ uint16_t bits16(__nv_bfloat16 x) { return __bfloat16_as_ushort(x); }
+template <typename T>
+__device__ __forceinline__ T from_bits16(uint16_t b);
+template <>
+__device__ __forceinline__ __half from_bits16<__half>(uint16_t b) { return __ushort_as_half(b); }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_bits16<__nv_bfloat16>(uint16_t b) { return __ushort_as_bfloat16(b); }
 
 // Row r's 16-byte piece k (k < 8) of a 128-byte-swizzled 128-row chunk.
 __device__ __forceinline__ uint32_t sw128_offset(int r, int k) { return r * 128 + ((k ^ (r & 7)) << 4); }
@@ -1004,6 +1010,7 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
             (p.mask_on && row_ok) ? p.mask + it.b * p.mask_b + it.n * p.mask_n + (int64_t)i * p.mask_i : nullptr;
 
         float m_run = -CUDART_INF_F, m_used = -CUDART_INF_F, l = 0.f;
+        uint32_t wnext[3];  // compressed bias: the warp's window values of the coming block
         for (int jb = tr.lo; jb <= tr.hi; ++jb) {
             if constexpr (kBias == 1) {
                 // the next block's bias row segment (256 bytes) on its way to L2
@@ -1081,9 +1088,9 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
             // rows: row i reads stored row 0 at column j + first - i, so the
             // warp needs 159 consecutive stored values per key block.  They
             // go to shared memory (in the bias buffers, unused for this bias
-            // form) as fp32 times log2(e), in four copies shifted by 0..3
-            // values, so that every row's 128 values are four-aligned runs
-            // of one copy.
+            // form) as fp32, in four copies shifted by 0..3 values, so that
+            // every row's 128 values are four-aligned runs of one copy.  Each
+            // lane loads the next block's values while this block runs.
             uint32_t wrow = 0;  // this thread's run in the warp's window (0: no window)
             if (kBias == 1 && sBias != nullptr && p.pse_rows1024) {
                 const int first = it.q_len - 1024;
@@ -1093,13 +1100,24 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                     const uint32_t wbase = smem_u32(sBias + (t * 4 + quad) * kWinBytes);
                     const T* srow = static_cast<const T*>(p.pse) + it.b * p.pse_b + it.n * p.pse_n;
                     const int col0 = j0 + first - w0 - 31;  // stored column of window value 0
+                    // two stored values per register (raw 16-bit), zero outside the keys
+                    auto window_pair = [&](int col_a, int col_b) -> uint32_t {
+                        const uint32_t a = (col_a >= 0 && col_a < it.kv_len) ? bits16(srow[col_a]) : 0u;
+                        const uint32_t b = (col_b >= 0 && col_b < it.kv_len) ? bits16(srow[col_b]) : 0u;
+                        return a | (b << 16);
+                    };
+                    if (jb == tr.lo) {
+#pragma unroll
+                        for (int m = 0; m < 3; ++m)
+                            wnext[m] = window_pair(col0 + lane + 64 * m, col0 + lane + 64 * m + 32);
+                    }
                     __syncwarp();  // every lane has read the previous block's window
 #pragma unroll
                     for (int m = 0; m < 6; ++m) {
                         const int x = lane + 32 * m;
                         if (x < kWinLen + 3) {
-                            const int col = col0 + x;
-                            const float g = (col >= 0 && col < it.kv_len) ? to_f(srow[col]) : 0.f;
+                            const uint32_t raw = (wnext[m >> 1] >> (16 * (m & 1))) & 0xffffu;
+                            const float g = to_f(from_bits16<T>(static_cast<uint16_t>(raw)));
 #pragma unroll
                             for (int k = 0; k < 4; ++k)
                                 if (x - k >= 0 && x - k < kWinLen)
@@ -1109,6 +1127,11 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                         }
                     }
                     __syncwarp();
+                    if (jb < tr.hi) {  // the next block's values, one block of keys on
+#pragma unroll
+                        for (int m = 0; m < 3; ++m)
+                            wnext[m] = window_pair(col0 + kTileN + lane + 64 * m, col0 + kTileN + lane + 64 * m + 32);
+                    }
                     const int x0 = 31 - lane;  // this row's first window value
                     wrow = wbase + ((x0 & 3) * kWinLen + (x0 & ~3)) * 4;
                 }
@@ -1151,8 +1174,10 @@ __device__ void run_softmax(const FaParams& p, Barriers& bars, const TicketSlots
                     }
                     // ALiBi terms are in log2 units; a bias tensor's are
                     // natural, so its scores stay natural (unit = log2 e)
+                    const float sm = kBias == 2 ? sl2 : abs_scale;
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) s[c16 + e] = fmaf(s[c16 + e], kBias == 2 ? sl2 : abs_scale, bias[e]);
+                    for (int e = 0; e < 16; e += 2)
+                        fma2(s[c16 + e], s[c16 + e + 1], s[c16 + e], s[c16 + e + 1], sm, sm, bias[e], bias[e + 1]);
                 }
             }
             if (tma_bias) {  // the buffer may be refilled
